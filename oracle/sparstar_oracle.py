@@ -1,0 +1,272 @@
+"""CPU oracle for SparSTAR's per-scale dynamic block-sparse attention (fp64, numpy).
+
+TEST INFRASTRUCTURE. Only the tests, the package's smoke check and the benchmark's CPU
+baseline may import this module. The CUDA library never calls it, and it imports nothing
+from the CUDA side: it takes plain arrays (bf16 bit patterns as uint16) and works in fp64.
+
+What it computes, per head, for one expensive scale. Source: the SparSTAR digest
+"SparSTAR的贡献：每尺度动态重建" (pchao.org), section 方法概览 ("method overview"), and the
+English abstract "SparSTAR: Sparse Attention for SpaceTime AutoRegressive Video Synthesis"
+(newx.sg), section Abstract:
+  1. split Q and the mixed KV context (text ‖ reference context ‖ current tokens) into
+     128-token blocks                                    (方法概览, bullet 块划分与聚合评分);
+  2. mean-pool each block                                 (same bullet: 对块内向量取均值);
+  3. score every (query block, key block) pair from the pooled vectors (same bullet);
+  4. keep the clip-aware conditioning blocks dense: text always, and in Clip 1 also the
+     image-pyramid blocks                                 (bullet clip感知保留策略);
+  5. fill each query-block row with a joint Top-K over the remaining key blocks
+     (方法概览 first paragraph: 对其余块联合Top-K选择), separately for every head
+     (bullet per-head动态掩码);
+  6. run forward-only attention over the kept blocks only (bullet FastFlex执行路径).
+The pages print no formulas, code or worked example for SparSTAR. Readings of the open
+points (all also listed in the design notes):
+  - score: S_ij = mean(q_i) . mean(k_j) / sqrt(d);
+  - budget: each row holds max(ceil(density * n_kv_blocks), n_forced) blocks ("literal");
+    the alternative "candidates" mode keeps ceil(density * n_candidates) Top-K blocks on
+    top of the forced ones;
+  - ties in the Top-K go to the lower block index;
+  - a ragged last block is pooled over its valid tokens only;
+  - blocks are counted globally over the concatenated KV; a block is forced when it holds
+    any forced (text, or Clip-1 context) token;
+  - no causal or intra-block mask; attention scale 1/sqrt(d).
+The retained attention mass used by the self-checks follows the block-energy definition of
+"Accelerating Text-to-Video Generation with Calibrated Sparse Attention" (papernotes.org),
+section 关键设计 1, eq. (5): the softmax mass that a query block's rows put on a set of key
+blocks, averaged over the rows.
+
+Every array here is fp64 except the uint16 inputs and int64 index outputs.
+"""
+from __future__ import annotations
+
+import math
+from typing import Sequence, Tuple
+
+import numpy as np
+
+BLOCK = 128  # 方法概览: "按128-token块划分"
+
+BUDGET_LITERAL = 0      # rows hold max(ceil(density * nkb), n_forced) blocks
+BUDGET_CANDIDATES = 1   # Top-K keeps ceil(density * n_candidates) non-forced blocks
+
+
+# --------------------------------------------------------------------------- inputs
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) exactly to fp64: a bf16 is the top half of an fp32."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    as_f32 = (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    return as_f32.astype(np.float64)
+
+
+# --------------------------------------------------------------------------- step 1
+
+def num_blocks(n_tokens: int, block: int = BLOCK) -> int:
+    """Number of `block`-token blocks covering n_tokens (the last one may be ragged)."""
+    return -(-int(n_tokens) // block)
+
+
+def block_token_range(j: int, n_tokens: int, block: int = BLOCK) -> Tuple[int, int]:
+    """[start, end) token range of block j; the last block stops at n_tokens."""
+    return j * block, min((j + 1) * block, n_tokens)
+
+
+def forced_block_count(n_text: int, n_ctx: int, clip: int, block: int = BLOCK) -> int:
+    """Blocks kept dense by the clip-aware rule (方法概览, bullet clip感知保留策略).
+
+    The KV context is text ‖ reference context ‖ current tokens, so the forced blocks are a
+    prefix of the KV blocks: the blocks holding text tokens, plus in Clip 1 the blocks
+    holding image-pyramid tokens. A block holding any forced token counts as forced.
+    """
+    forced_tokens = n_text + (n_ctx if clip == 1 else 0)
+    return num_blocks(forced_tokens, block)
+
+
+def ceil_exact(x: float) -> int:
+    """ceil with a 1e-9 guard so that a product such as 0.1875 * 16 = 3.0 stays 3."""
+    return int(math.ceil(x - 1e-9))
+
+
+def row_budget(nkb: int, n_forced: int, density: float, mode: int = BUDGET_LITERAL) -> Tuple[int, int]:
+    """(K_total, K_topk): blocks kept per query-block row, and how many of them Top-K picks.
+
+    Literal reading: fill each row to ceil(density * nkb) blocks, never fewer than the
+    forced ones. Candidates reading: Top-K picks ceil(density * n_candidates) of the
+    non-forced blocks. Both are clipped to what exists.
+    """
+    n_forced = min(n_forced, nkb)
+    n_cand = nkb - n_forced
+    if mode == BUDGET_LITERAL:
+        k_total = min(max(ceil_exact(density * nkb), n_forced), nkb)
+        k_topk = k_total - n_forced
+    elif mode == BUDGET_CANDIDATES:
+        k_topk = min(ceil_exact(density * n_cand), n_cand)
+        k_total = n_forced + k_topk
+    else:
+        raise ValueError(f"unknown budget mode {mode}")
+    return k_total, k_topk
+
+
+# --------------------------------------------------------------------------- step 2
+
+def pool_blocks(x: np.ndarray, block: int = BLOCK) -> np.ndarray:
+    """Mean of the token vectors inside each block, [N, d] -> [nb, d] (方法概览: 对块内向量取均值).
+
+    A ragged last block is averaged over its valid tokens only.
+    """
+    n, d = x.shape
+    nb = num_blocks(n, block)
+    out = np.zeros((nb, d), dtype=np.float64)
+    for j in range(nb):
+        s, e = block_token_range(j, n, block)
+        out[j] = x[s:e].sum(axis=0) / (e - s)
+    return out
+
+
+# --------------------------------------------------------------------------- step 3
+
+def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Aggregate compatibility S_ij = qbar_i . kbar_j / sqrt(d), [nqb, nkb] (方法概览)."""
+    d = qbar.shape[1]
+    return (qbar @ kbar.T) / math.sqrt(d)
+
+
+# --------------------------------------------------------------------------- steps 4-5
+
+def _order_scores(s: np.ndarray) -> np.ndarray:
+    # -0.0 and +0.0 are the same score; NaN (never produced from finite inputs) ranks last.
+    s = np.where(np.isnan(s), -np.inf, s)
+    return s + 0.0
+
+
+def select_rows(S: np.ndarray, n_forced: int, k_topk: int) -> np.ndarray:
+    """Kept KV blocks of each query-block row, ascending (方法概览: clip-aware retention + joint Top-K).
+
+    S is [nqb, nkb]. The forced blocks 0..n_forced-1 are always kept. The K_topk
+    highest-scoring remaining blocks join them; among equal scores the lower block index
+    comes first. The ranking is one library sort per row on the key (-score, index).
+    """
+    nqb, nkb = S.shape
+    n_forced = min(n_forced, nkb)
+    cand = _order_scores(S[:, n_forced:])
+    index = np.broadcast_to(np.arange(n_forced, nkb), cand.shape)
+    order = np.lexsort((index, -cand), axis=-1)          # primary key last: -score, then index
+    chosen = np.sort(order[:, :k_topk] + n_forced, axis=1)
+    forced = np.broadcast_to(np.arange(n_forced), (nqb, n_forced))
+    return np.concatenate([forced, chosen], axis=1).astype(np.int64)
+
+
+def select_row(scores_row: np.ndarray, n_forced: int, k_topk: int) -> np.ndarray:
+    """One row of select_rows."""
+    return select_rows(np.asarray(scores_row, dtype=np.float64)[None, :], n_forced, k_topk)[0]
+
+
+def select_head(q: np.ndarray, k: np.ndarray, n_text: int, n_ctx: int, clip: int,
+                density: float, mode: int = BUDGET_LITERAL, block: int = BLOCK):
+    """One head's block mask. q [Nq,d], k [Nkv,d] fp64 -> (rows [nqb, K_total] int64, S [nqb, nkb])."""
+    nkb = num_blocks(k.shape[0], block)
+    n_forced = min(forced_block_count(n_text, n_ctx, clip, block), nkb)
+    k_total, k_topk = row_budget(nkb, n_forced, density, mode)
+    S = block_scores(pool_blocks(q, block), pool_blocks(k, block))
+    return select_rows(S, n_forced, k_topk), S
+
+
+def select(q_bits: np.ndarray, k_bits: np.ndarray, n_text: int, n_ctx: int, clip: int,
+           density: float, mode: int = BUDGET_LITERAL, block: int = BLOCK):
+    """All heads (per-head masks, bullet per-head动态掩码). Inputs are bf16 bits [H,N,d].
+
+    Returns (idx [H, nqb, K_total] int64, scores [H, nqb, nkb] fp64).
+    """
+    H = q_bits.shape[0]
+    idx, scores = [], []
+    for h in range(H):
+        rows, S = select_head(bf16_bits_to_f64(q_bits[h]), bf16_bits_to_f64(k_bits[h]),
+                              n_text, n_ctx, clip, density, mode, block)
+        idx.append(rows)
+        scores.append(S)
+    return np.stack(idx), np.stack(scores)
+
+
+# --------------------------------------------------------------------------- step 6
+
+def kept_token_index(kept_blocks: Sequence[int], n_kv: int, block: int = BLOCK) -> np.ndarray:
+    """Token positions of the kept KV blocks (valid tokens only)."""
+    parts = [np.arange(*block_token_range(int(j), n_kv, block)) for j in kept_blocks]
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+
+
+def attend_rows(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, tokens: np.ndarray,
+                sm_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention of q_rows over the listed KV tokens (bullet FastFlex执行路径).
+
+    logits l_u = sm_scale * q . k_u; o = sum_u softmax(l)_u v_u; lse = log sum_u exp(l_u).
+    Returns (o [n, d], lse [n]) in fp64.
+    """
+    logits = (q_rows @ k[tokens].T) * sm_scale
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    z = e.sum(axis=1, keepdims=True)
+    o = (e @ v[tokens]) / z
+    lse = (m + np.log(z))[:, 0]
+    return o, lse
+
+
+def block_sparse_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,
+                           qblocks: Sequence[int], sm_scale: float | None = None,
+                           block: int = BLOCK):
+    """Attention of the listed query blocks over their kept KV blocks (one head, fp64 inputs).
+
+    rows[i] is the kept-block list of query block i (entries < 0 are ignored). Returns a
+    list of (o [n_i, d], lse [n_i]) in the order of qblocks.
+    """
+    d = q.shape[1]
+    scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    out = []
+    for i in qblocks:
+        s, e = block_token_range(int(i), q.shape[0], block)
+        kept = [int(j) for j in rows[int(i)] if j >= 0]
+        out.append(attend_rows(q[s:e], k, v, kept_token_index(kept, k.shape[0], block), scale))
+    return out
+
+
+def dense_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, qblocks: Sequence[int],
+                    sm_scale: float | None = None, block: int = BLOCK):
+    """Attention over every KV token (the density = 1 case), same return as above."""
+    nkb = num_blocks(k.shape[0], block)
+    all_rows = np.tile(np.arange(nkb), (num_blocks(q.shape[0], block), 1))
+    return block_sparse_attention(q, k, v, all_rows, qblocks, sm_scale, block)
+
+
+def retained_mass(lse_kept: np.ndarray, lse_dense: np.ndarray) -> np.ndarray:
+    """Per query row, the dense softmax mass on the kept tokens: exp(lse_kept - lse_dense).
+
+    Averaged over the rows of a query block this is the block energy of eq. (5) of the
+    CalibAtt notes, summed over the kept key blocks.
+    """
+    return np.exp(lse_kept - lse_dense)
+
+
+def block_energy(q: np.ndarray, k: np.ndarray, qblock: int, key_blocks: Sequence[int],
+                 sm_scale: float | None = None, block: int = BLOCK) -> float:
+    """Eq. (5) of the CalibAtt notes, summed over key_blocks: (1/n_i) sum_t sum_u P_tu.
+
+    P is the dense softmax over all KV tokens; rows t are the valid tokens of query block
+    `qblock` (n_i of them) and columns u the valid tokens of key_blocks.
+    """
+    d = q.shape[1]
+    scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    s, e = block_token_range(qblock, q.shape[0], block)
+    logits = (q[s:e] @ k.T) * scale
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    p /= p.sum(axis=1, keepdims=True)
+    cols = kept_token_index(key_blocks, k.shape[0], block)
+    return float(p[:, cols].sum() / (e - s))
+
+
+__all__ = [
+    "BLOCK", "BUDGET_LITERAL", "BUDGET_CANDIDATES", "bf16_bits_to_f64", "num_blocks",
+    "block_token_range", "forced_block_count", "row_budget", "pool_blocks", "block_scores",
+    "select_rows", "select_row", "select_head", "select", "kept_token_index", "attend_rows",
+    "block_sparse_attention", "dense_attention", "retained_mass", "block_energy",
+]
+
