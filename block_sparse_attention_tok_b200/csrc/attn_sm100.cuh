@@ -1,0 +1,452 @@
+// Forward-only block-sparse flash attention over kept 128x128 tiles, for sm_100a.
+//
+// Computes the attention of the SparSTAR digest ("SparSTAR的贡献：每尺度动态重建", pchao.org),
+// section 方法概览, bullet FastFlex执行路径: only the KV blocks listed for a query block are
+// visited, with an online softmax across them. The pages' executor (a FlexAttention
+// variant) is prior art for other hardware; this kernel is written for Blackwell:
+//
+//   * persistent grid, one CTA per SM; a CTA owns two "slots", each working through its own
+//     sequence of (head, query block) items, so the softmax of one slot overlaps the tensor
+//     core work of the other;
+//   * warp 8 (TMA): loads the slot's 128xd Q tile once per item and, per kept block, the K
+//     and V tiles into a ring of shared-memory stages (128-byte swizzle, no multicast);
+//   * warp 9 (MMA, one thread): S = Q K^T into tensor memory (tcgen05.mma, M=128, N=128,
+//     K=16 steps), then O += P V with P read from tensor memory;
+//   * warps 0-3 / 4-7 (softmax of slot 0 / 1, one thread per query row): tcgen05.ld of the
+//     S row, masking of a ragged last KV block, running max with a lazy rescale (the
+//     running max only moves when a tile's max exceeds it by more than 8 in log2 units,
+//     so P stays <= 256 and O is rarely rescaled), exp2, row sum, bf16 P written back over
+//     S with tcgen05.st, and the epilogue O / l -> bf16, lse = ln 2 * (m + log2 l).
+//
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [384,384+d).
+// P of slot s overwrites the first 64 columns of S_s as packed bf16 pairs.
+//
+// Ordering: tcgen05.mma ops issued by one thread execute in order, and a tcgen05.commit
+// arrives once all earlier ops of that thread are done. S_s(n+1) is issued after
+// PV_s(n), so when the softmax sees S_s(n+1) complete, PV_s(n) is complete too: it may
+// rescale O_s and overwrite P_s without further waits.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace sparstar {
+
+template <int D>
+struct AttnConfig {
+  static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+  static constexpr int kRows = 128;                    // query rows per tile (one query block)
+  static constexpr int kCols = 128;                    // KV tokens per tile (one KV block)
+  static constexpr int kChunks = D / 64;               // 128-byte swizzle chunks per row
+  static constexpr uint32_t kChunkBytes = 128 * 128;   // 128 rows x 128 bytes
+  static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring depth
+  static constexpr int kSlots = 2;
+  static constexpr int kThreads = 320;                 // 8 softmax warps + TMA warp + MMA warp
+  static constexpr int kLoadWarp = 8;
+  static constexpr int kMmaWarp = 9;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemS = 0;                // + 128 * slot
+  static constexpr uint32_t kTmemO = 256;              // + 128 * slot
+  static constexpr uint32_t kSmemBytes = 1024 /*align*/ + kSlots * kTileBytes + kStages * kTileBytes + 512;
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+};
+
+struct AttnParams {
+  const int32_t* idx;   // [H, nqb, kmax]
+  const int32_t* cnt;   // [H, nqb]
+  __nv_bfloat16* o;     // [H, Nq, D]
+  float* lse;           // [H, Nq] or nullptr
+  unsigned* status;     // device status word
+  int64_t n_q, n_kv;
+  int nqb, nkb, kmax, n_items;
+  float scale_log2;     // sm_scale * log2(e)
+};
+
+// Work sequence of one slot: items slot_id, slot_id + stride, ... (head-major order).
+struct SlotSeq {
+  int item;     // current item, or -1 when the slot is finished
+  int ntiles;   // kept blocks of the current item
+  int n;        // current tile within the item
+  int k;        // number of items started before the current one
+  int h, qb;
+};
+
+__device__ __forceinline__ int clamp_count(int c, int kmax, unsigned* status, bool report) {
+  if (c < 1 || c > kmax) {
+    if (report) atomicOr(status, kStatusBounds);
+    c = c < 1 ? 1 : kmax;
+  }
+  return c;
+}
+
+__device__ __forceinline__ int clamp_block(int j, int nkb, unsigned* status, bool report) {
+  if (j < 0 || j >= nkb) {
+    if (report) atomicOr(status, kStatusBounds);
+    j = j < 0 ? 0 : nkb - 1;
+  }
+  return j;
+}
+
+__device__ __forceinline__ void seq_begin(SlotSeq& s, const AttnParams& p, bool report) {
+  if (s.item >= p.n_items) {
+    s.item = -1;
+    return;
+  }
+  s.h = s.item / p.nqb;
+  s.qb = s.item - s.h * p.nqb;
+  s.ntiles = clamp_count(__ldg(p.cnt + s.item), p.kmax, p.status, report);
+  s.n = 0;
+}
+
+__device__ __forceinline__ void seq_init(SlotSeq& s, int slot_id, const AttnParams& p, bool report) {
+  s.item = slot_id;
+  s.k = 0;
+  seq_begin(s, p, report);
+}
+
+// Advance to the next tile; returns true when a new item started.
+__device__ __forceinline__ bool seq_next(SlotSeq& s, int stride, const AttnParams& p, bool report) {
+  if (++s.n < s.ntiles) return false;
+  s.item += stride;
+  ++s.k;
+  seq_begin(s, p, report);
+  return true;
+}
+
+__device__ __forceinline__ int seq_block(const SlotSeq& s, const AttnParams& p, bool report) {
+  const int j = __ldg(p.idx + static_cast<int64_t>(s.item) * p.kmax + s.n);
+  return clamp_block(j, p.nkb, p.status, report);
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
+    attn_sparse_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnConfig<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* q_tile = smem;                                   // [slot] kTileBytes each
+  uint8_t* ring = smem + C::kSlots * C::kTileBytes;         // [stage] kTileBytes each
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::kStages * C::kTileBytes);
+  uint64_t* full = bars;                      // [kStages] TMA -> MMA
+  uint64_t* empty = full + C::kStages;        // [kStages] MMA -> TMA
+  uint64_t* q_full = empty + C::kStages;      // [2]
+  uint64_t* q_empty = q_full + 2;             // [2]
+  uint64_t* s_full = q_empty + 2;             // [2] MMA -> softmax
+  uint64_t* p_full = s_full + 2;              // [2] softmax -> MMA
+  uint64_t* o_full = p_full + 2;              // [2] MMA -> softmax (end of item)
+  uint64_t* drain = o_full + 2;               // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * C::kSlots;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_full[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == C::kLoadWarp && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == C::kLoadWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      SlotSeq seq[2];
+      seq_init(seq[0], blockIdx.x * 2 + 0, p, true);
+      seq_init(seq[1], blockIdx.x * 2 + 1, p, true);
+      uint32_t ring_it = 0;
+      int last_q_k[2] = {-1, -1};
+      bool ok = true;
+
+      auto load_q = [&](int s) -> bool {
+        if (!mbar_wait(&q_empty[s], (seq[s].k & 1) ^ 1, abort_flag, p.status)) return false;
+        mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
+        const uint32_t dst = smem_u32(q_tile + s * C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(dst + c * C::kChunkBytes, &tm_q, &q_full[s], c * 64, seq[s].qb * 128, seq[s].h);
+        last_q_k[s] = seq[s].k;
+        return true;
+      };
+      auto load_kv = [&](int s, const CUtensorMap* map) -> bool {
+        const int j = seq_block(seq[s], p, true);
+        const uint32_t stage = ring_it % C::kStages;
+        const uint32_t phase = (ring_it / C::kStages) & 1u;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
+        mbar_arrive_expect_tx(&full[stage], C::kTileBytes);
+        const uint32_t dst = smem_u32(ring + stage * C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(dst + c * C::kChunkBytes, map, &full[stage], c * 64, j * 128, seq[s].h);
+        ++ring_it;
+        return true;
+      };
+
+      for (int s = 0; s < 2 && ok; ++s)
+        if (seq[s].item >= 0) ok = load_q(s) && load_kv(s, &tm_k);
+      while (ok && (seq[0].item >= 0 || seq[1].item >= 0)) {
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (seq[s].item < 0) continue;
+          ok = load_kv(s, &tm_v);
+          if (!ok) break;
+          const bool new_item = seq_next(seq[s], stride, p, true);
+          if (seq[s].item < 0) continue;
+          if (new_item) ok = load_q(s);
+          if (ok) ok = load_kv(s, &tm_k);
+        }
+      }
+      // Drain: wait until every load issued into a stage or Q buffer has landed, so no TMA
+      // write is in flight when the CTA exits (matters only after an abort).
+      for (uint32_t st = 0; st < C::kStages; ++st) {
+        if (ring_it > st) {
+          const uint32_t last_use = ring_it - 1 - ((ring_it - 1 - st) % C::kStages);
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[st], (last_use / C::kStages) & 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+      for (int s = 0; s < 2; ++s) {
+        if (last_q_k[s] >= 0) {
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&q_full[s], last_q_k[s] & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      SlotSeq seq[2];
+      seq_init(seq[0], blockIdx.x * 2 + 0, p, false);
+      seq_init(seq[1], blockIdx.x * 2 + 1, p, false);
+      uint32_t ring_it = 0;
+      uint32_t tiles[2] = {0u, 0u};
+      bool ok = true;
+
+      auto issue_s = [&](int s) -> bool {
+        if (seq[s].n == 0 && !mbar_wait(&q_full[s], seq[s].k & 1, abort_flag, p.status)) return false;
+        const uint32_t stage = ring_it % C::kStages;
+        if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(q_tile + s * C::kTileBytes);
+        const uint32_t ka = smem_u32(ring + stage * C::kTileBytes);
+        const uint32_t d_tmem = tmem_base + C::kTmemS + 128u * s;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), C::kIdescQK,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[stage]);
+        mma_commit(&s_full[s]);
+        if (seq[s].n == seq[s].ntiles - 1) mma_commit(&q_empty[s]);
+        ++ring_it;
+        return true;
+      };
+      auto issue_pv = [&](int s) -> bool {
+        if (!mbar_wait(&p_full[s], tiles[s] & 1u, abort_flag, p.status)) return false;
+        ++tiles[s];
+        const uint32_t stage = ring_it % C::kStages;
+        if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t va = smem_u32(ring + stage * C::kTileBytes);
+        const uint32_t d_tmem = tmem_base + C::kTmemO + 128u * s;
+        const uint32_t a_tmem = tmem_base + C::kTmemS + 128u * s;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // P columns: 16 bf16 per K step = 8 packed 32-bit columns.
+          // V tile is MN-major for this MMA: 64-element chunks of d at 16 KB (LBO), 8-row
+          // groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
+          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
+                 (seq[s].n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[stage]);
+        if (seq[s].n == seq[s].ntiles - 1) mma_commit(&o_full[s]);
+        ++ring_it;
+        return true;
+      };
+
+      for (int s = 0; s < 2 && ok; ++s)
+        if (seq[s].item >= 0) ok = issue_s(s);
+      while (ok && (seq[0].item >= 0 || seq[1].item >= 0)) {
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (seq[s].item < 0) continue;
+          ok = issue_pv(s);
+          if (!ok) break;
+          seq_next(seq[s], stride, p, false);
+          if (seq[s].item < 0) continue;
+          ok = issue_s(s);
+        }
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      mma_commit(drain);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int s = warp >> 2;          // slot
+    const int wq = warp & 3;          // TMEM lane quarter
+    const int row = wq * 32 + lane;   // query row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem_base + lane_off + C::kTmemS + 128u * s;
+    const uint32_t t_o = tmem_base + lane_off + C::kTmemO + 128u * s;
+    SlotSeq seq;
+    seq_init(seq, blockIdx.x * 2 + s, p, false);
+    uint32_t tiles = 0, items = 0;
+    bool ok = true;
+    while (ok && seq.item >= 0) {
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int n = 0; n < seq.ntiles && ok; ++n) {
+        seq.n = n;
+        const int j = seq_block(seq, p, false);
+        const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * 128) : 128;
+        if (!mbar_wait(&s_full[s], tiles & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        ++tiles;
+        tc_fence_after();
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r[c]);
+        tmem_wait_ld();
+        if (n_valid < 128) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * c + e >= n_valid) r[c][e] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[c][e]));
+        const float mx_scaled = mx * p.scale_log2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx_scaled > m_run + 8.f) {
+          alpha = ex2_approx(m_run - mx_scaled);  // m_run = -inf on the first tile -> 0
+          l_run *= alpha;
+          m_run = mx_scaled;
+          rescale = (n > 0);
+        }
+        float rowsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e]), p.scale_log2, -m_run));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e + 1]), p.scale_log2, -m_run));
+            rowsum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[c][e] = pk[e];
+        }
+        l_run += rowsum;
+        if (rescale) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + 32 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(t_o + 32 * c, ov);
+          }
+        }
+        // P: 128 bf16 = 64 packed columns over the start of S.
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            pk[e] = r[2 * c][e];
+            pk[16 + e] = r[2 * c + 1][e];
+          }
+          tmem_st32(t_s + 32 * c, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[s]);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16, lse
+      if (!mbar_wait(&o_full[s], items & 1u, abort_flag, p.status)) break;
+      ++items;
+      tc_fence_after();
+      const int64_t t = static_cast<int64_t>(seq.qb) * 128 + row;
+      const bool valid = t < p.n_q;
+      const float inv_l = 1.f / l_run;
+      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(seq.h) * p.n_q + t) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(t_o + 32 * c, ov);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[static_cast<int64_t>(seq.h) * p.n_q + t] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+      tc_fence_before();
+      seq.n = seq.ntiles - 1;
+      seq_next(seq, stride, p, false);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace sparstar

@@ -1,0 +1,323 @@
+// Host side of the C ABI declared in include/sparstar.h, and the single translation unit
+// that instantiates every kernel of the library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sparstar.h"
+#include "attn_sm100.cuh"
+#include "select.cuh"
+
+namespace sparstar {
+
+// Per-device status word: bit kStatusTimeout / kStatusBounds, set by kernels, read by
+// sparstar_device_status(). A __device__ variable exists once per device that loads the
+// library, so no allocation is needed.
+__device__ unsigned g_status = 0u;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxCandidates = 16384;  // Top-K keys held in shared memory (64 KB)
+
+struct DeviceInfo {
+  bool ready = false;
+  int major = 0, minor = 0, sms = 0;
+  unsigned* status = nullptr;
+  bool attrs_set = false;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SPARSTAR_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SPARSTAR_ERR_CUDA;
+    d.major = prop.major;
+    d.minor = prop.minor;
+    d.sms = prop.multiProcessorCount;
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_status) != cudaSuccess) return SPARSTAR_ERR_CUDA;
+    d.status = static_cast<unsigned*>(sym);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return SPARSTAR_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return SPARSTAR_OK;
+}
+
+int set_kernel_attrs(DeviceInfo* d) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (d->attrs_set) return SPARSTAR_OK;
+  bool ok = true;
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnConfig<128>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnConfig<64>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * 64 * (128 + 4) * 4) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kMaxCandidates * 4)) == cudaSuccess;
+  if (!ok) return SPARSTAR_ERR_CUDA;
+  d->attrs_set = true;
+  return SPARSTAR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_blocks(int64_t n) { return (n + SPARSTAR_BLOCK - 1) / SPARSTAR_BLOCK; }
+
+// ceil(x) with a 1e-9 guard, so that a product such as 0.1875 * 16 = 3.0 stays 3.
+int64_t ceil_guarded(double x) { return static_cast<int64_t>(std::ceil(x - 1e-9)); }
+
+bool valid_segments(const sparstar_segments& s) { return s.n_text >= 0 && s.n_ctx >= 0 && s.n_cur >= 0; }
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+struct Workspace {
+  size_t qbar, kbar, scores, total;
+};
+
+Workspace workspace_layout(int heads, int64_t nqb, int64_t nkb, int d, bool need_scores) {
+  Workspace w;
+  w.qbar = 0;
+  w.kbar = align256(static_cast<size_t>(heads) * nqb * d * sizeof(float));
+  w.scores = w.kbar + align256(static_cast<size_t>(heads) * nkb * d * sizeof(float));
+  w.total = w.scores + (need_scores ? align256(static_cast<size_t>(heads) * nqb * nkb * sizeof(float)) : 0);
+  return w;
+}
+
+int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d) {
+  // 3-D view [heads][rows][d] of bf16; box = 64 elements x 128 rows x 1 head, 128B swizzle.
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SPARSTAR_OK : SPARSTAR_ERR_CUDA;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ERR_CUDA; }
+
+}  // namespace
+}  // namespace sparstar
+
+using namespace sparstar;
+
+extern "C" {
+
+int sparstar_abi_version(void) { return SPARSTAR_ABI_VERSION; }
+
+const char* sparstar_strerror(int code) {
+  switch (code) {
+    case SPARSTAR_OK: return "ok";
+    case SPARSTAR_ERR_ARG: return "invalid argument";
+    case SPARSTAR_ERR_UNSUPPORTED: return "unsupported head_dim, device or size";
+    case SPARSTAR_ERR_WORKSPACE: return "workspace missing or too small";
+    case SPARSTAR_ERR_CUDA: return "CUDA call failed";
+    case SPARSTAR_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case SPARSTAR_ERR_DEVICE_BOUNDS: return "device clamped an out-of-range index or count";
+    default: return "unknown status";
+  }
+}
+
+int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double density, int budget_mode,
+                       sparstar_plan* out) {
+  if (out == nullptr || n_q < 0 || !valid_segments(seg) || clip < 1 || !(density > 0.0) || !(density <= 1.0) ||
+      (budget_mode != SPARSTAR_BUDGET_LITERAL && budget_mode != SPARSTAR_BUDGET_CANDIDATES))
+    return SPARSTAR_ERR_ARG;
+  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
+  if (n_kv < 1) return SPARSTAR_ERR_ARG;
+  sparstar_plan p;
+  p.nqb = ceil_blocks(n_q);
+  p.nkb = ceil_blocks(n_kv);
+  const int64_t forced_tokens = seg.n_text + (clip == 1 ? seg.n_ctx : 0);
+  p.n_forced = ceil_blocks(forced_tokens);
+  if (p.n_forced > p.nkb) p.n_forced = p.nkb;
+  p.n_cand = p.nkb - p.n_forced;
+  int64_t k_total, k_topk;
+  if (budget_mode == SPARSTAR_BUDGET_LITERAL) {
+    k_total = ceil_guarded(density * static_cast<double>(p.nkb));
+    if (k_total < p.n_forced) k_total = p.n_forced;
+    if (k_total > p.nkb) k_total = p.nkb;
+    k_topk = k_total - p.n_forced;
+  } else {
+    k_topk = ceil_guarded(density * static_cast<double>(p.n_cand));
+    if (k_topk > p.n_cand) k_topk = p.n_cand;
+    if (k_topk < 0) k_topk = 0;
+    k_total = p.n_forced + k_topk;
+  }
+  if (k_total > INT32_MAX) return SPARSTAR_ERR_UNSUPPORTED;
+  p.k_total = static_cast<int32_t>(k_total);
+  p.k_topk = static_cast<int32_t>(k_topk);
+  *out = p;
+  return SPARSTAR_OK;
+}
+
+int sparstar_workspace_size(int heads, int64_t n_q, sparstar_segments seg, int head_dim, size_t* bytes) {
+  if (bytes == nullptr || heads < 1 || n_q < 0 || !valid_segments(seg)) return SPARSTAR_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
+  if (n_kv < 1) return SPARSTAR_ERR_ARG;
+  *bytes = workspace_layout(heads, ceil_blocks(n_q), ceil_blocks(n_kv), head_dim, true).total;
+  return SPARSTAR_OK;
+}
+
+int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparstar_segments seg, int head_dim,
+                    int clip, double density, int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
+                    float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+  sparstar_plan plan;
+  int rc = sparstar_make_plan(n_q, seg, clip, density, budget_mode, &plan);
+  if (rc != SPARSTAR_OK) return rc;
+  if (heads < 1) return SPARSTAR_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  if (n_q == 0) return SPARSTAR_OK;
+  if (q == nullptr || k == nullptr || idx == nullptr || cnt == nullptr || !aligned16(q) || !aligned16(k) ||
+      (scores != nullptr && !aligned16(scores)) || kmax < plan.k_total)
+    return SPARSTAR_ERR_ARG;
+  const int64_t rows = static_cast<int64_t>(heads) * plan.nqb;
+  if (rows > INT32_MAX || static_cast<int64_t>(heads) * (plan.nqb + plan.nkb) > INT32_MAX ||
+      plan.nqb > 65535 * 64LL || plan.n_cand > kMaxCandidates || heads > 65535)
+    return SPARSTAR_ERR_UNSUPPORTED;
+  const bool needs_scores = plan.k_topk > 0 && plan.k_topk < plan.n_cand;
+  const bool compute_scores = needs_scores || scores != nullptr;
+  const Workspace ws = workspace_layout(heads, plan.nqb, plan.nkb, head_dim, scores == nullptr);
+  if (compute_scores && (workspace == nullptr || workspace_bytes < ws.total ||
+                         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return SPARSTAR_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != SPARSTAR_OK) return rc;
+  if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
+  const int nqb = static_cast<int>(plan.nqb), nkb = static_cast<int>(plan.nkb);
+
+  if (compute_scores) {
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    float* qbar = reinterpret_cast<float*>(wsb + ws.qbar);
+    float* kbar = reinterpret_cast<float*>(wsb + ws.kbar);
+    float* S = scores != nullptr ? scores : reinterpret_cast<float*>(wsb + ws.scores);
+    const unsigned pool_grid = static_cast<unsigned>(heads) * static_cast<unsigned>(nqb + nkb);
+    const dim3 sgrid((nkb + 63) / 64, (nqb + 63) / 64, heads);
+    const float inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(head_dim));
+    if (head_dim == 128) {
+      pool_kernel<128><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, qbar,
+                                                  kbar);
+      score_kernel<128><<<sgrid, 256, 2 * 64 * (128 + 4) * 4, st>>>(qbar, kbar, nqb, nkb, inv_sqrt_d, S);
+    } else {
+      pool_kernel<64><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                                 static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, qbar,
+                                                 kbar);
+      score_kernel<64><<<sgrid, 256, 2 * 64 * (64 + 4) * 4, st>>>(qbar, kbar, nqb, nkb, inv_sqrt_d, S);
+    }
+    if ((rc = launch_status()) != SPARSTAR_OK) return rc;
+    if (needs_scores) {
+      topk_kernel<<<static_cast<unsigned>(rows), 128, static_cast<size_t>(plan.n_cand) * 4, st>>>(
+          S, nkb, static_cast<int>(plan.n_forced), plan.k_topk, idx, cnt, kmax);
+      return launch_status();
+    }
+  }
+  fill_kernel<<<static_cast<unsigned>(rows), 128, 0, st>>>(plan.k_total, idx, cnt, kmax);
+  return launch_status();
+}
+
+int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_t n_q, int64_t n_kv, int head_dim,
+                  const int32_t* idx, const int32_t* cnt, int32_t kmax, float sm_scale, void* o, float* lse,
+                  void* stream) {
+  if (heads < 1 || n_q < 0 || n_kv < 1 || kmax < 1) return SPARSTAR_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SPARSTAR_ERR_ARG;
+  if (n_q == 0) return SPARSTAR_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || idx == nullptr || cnt == nullptr ||
+      !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+    return SPARSTAR_ERR_ARG;
+  const int64_t nqb = ceil_blocks(n_q), nkb = ceil_blocks(n_kv);
+  if (static_cast<int64_t>(heads) * nqb > INT32_MAX / 2 || n_q > INT32_MAX || n_kv > INT32_MAX || nkb > INT32_MAX)
+    return SPARSTAR_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;
+  if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, n_q, heads, head_dim) != SPARSTAR_OK || make_map(&tk, k, n_kv, heads, head_dim) != SPARSTAR_OK ||
+      make_map(&tv, v, n_kv, heads, head_dim) != SPARSTAR_OK)
+    return SPARSTAR_ERR_CUDA;
+  AttnParams p;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = dev->status;
+  p.n_q = n_q;
+  p.n_kv = n_kv;
+  p.nqb = static_cast<int>(nqb);
+  p.nkb = static_cast<int>(nkb);
+  p.kmax = kmax;
+  p.n_items = static_cast<int>(heads * nqb);
+  const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int slots_needed = (p.n_items + 1) / 2;
+  const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128)
+    attn_sparse_kernel<128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
+  else
+    attn_sparse_kernel<64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+int sparstar_forward(const void* q, const void* k, const void* v, int heads, int64_t n_q, sparstar_segments seg,
+                     int head_dim, int clip, double density, int budget_mode, float sm_scale, int32_t* idx,
+                     int32_t* cnt, int32_t kmax, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (v == nullptr || o == nullptr) return SPARSTAR_ERR_ARG;
+  int rc = sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
+                           workspace, workspace_bytes, stream);
+  if (rc != SPARSTAR_OK) return rc;
+  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
+  return sparstar_attn(q, k, v, heads, n_q, n_kv, head_dim, idx, cnt, kmax, sm_scale, o, lse, stream);
+}
+
+int sparstar_device_status(void* stream, int clear) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SPARSTAR_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, dev->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return SPARSTAR_ERR_CUDA;
+  if (clear && word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return SPARSTAR_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) return SPARSTAR_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusBounds) return SPARSTAR_ERR_DEVICE_BOUNDS;
+  return SPARSTAR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,213 @@
+"""Python binding of the C-ABI library (libsparstar.so): argument marshalling only.
+
+Every step of the path (pooling, scoring, Top-K, attention) runs in the library's CUDA
+kernels. Torch is used to allocate device memory and to name the current stream. The
+binding raises if the library is missing: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from . import _build
+
+BLOCK = 128
+BUDGET_LITERAL = 0
+BUDGET_CANDIDATES = 1
+
+OK = 0
+ERR_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_WORKSPACE = 3
+ERR_CUDA = 4
+ERR_DEVICE_TIMEOUT = 5
+ERR_DEVICE_BOUNDS = 6
+
+# Every function the header declares, with (restype, argtypes).
+_c = ctypes
+_SIGNATURES = {}
+
+
+class Segments(ctypes.Structure):
+    _fields_ = [("n_text", ctypes.c_int64), ("n_ctx", ctypes.c_int64), ("n_cur", ctypes.c_int64)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("nqb", ctypes.c_int64), ("nkb", ctypes.c_int64), ("n_forced", ctypes.c_int64),
+                ("n_cand", ctypes.c_int64), ("k_total", ctypes.c_int32), ("k_topk", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: int(getattr(self, f)) for f, _ in self._fields_}
+
+
+_SIGNATURES.update({
+    "sparstar_abi_version": (_c.c_int, []),
+    "sparstar_strerror": (_c.c_char_p, [_c.c_int]),
+    "sparstar_make_plan": (_c.c_int, [_c.c_int64, Segments, _c.c_int, _c.c_double, _c.c_int, _c.POINTER(Plan)]),
+    "sparstar_workspace_size": (_c.c_int, [_c.c_int, _c.c_int64, Segments, _c.c_int, _c.POINTER(_c.c_size_t)]),
+    "sparstar_select": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments, _c.c_int, _c.c_int,
+                                   _c.c_double, _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p,
+                                   _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "sparstar_attn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                 _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_float, _c.c_void_p, _c.c_void_p,
+                                 _c.c_void_p]),
+    "sparstar_forward": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments, _c.c_int,
+                                    _c.c_int, _c.c_double, _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p,
+                                    _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "sparstar_device_status": (_c.c_int, [_c.c_void_p, _c.c_int]),
+})
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+class SparstarError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+def lib_path() -> str:
+    return _build.LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load libsparstar.so from the package directory (raises if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with __graft_entry__.build() "
+                               "(there is no CPU fallback)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def strerror(code: int) -> str:
+    return load().sparstar_strerror(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SparstarError(code, where)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) or None
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else int(t.data_ptr()) or None
+
+
+def make_plan(n_q: int, n_text: int, n_ctx: int, n_cur: int, clip: int, density: float,
+              budget_mode: int = BUDGET_LITERAL) -> Plan:
+    plan = Plan()
+    _check(load().sparstar_make_plan(int(n_q), Segments(n_text, n_ctx, n_cur), int(clip), float(density),
+                                     int(budget_mode), ctypes.byref(plan)), "sparstar_make_plan")
+    return plan
+
+
+def workspace_size(heads: int, n_q: int, n_text: int, n_ctx: int, n_cur: int, head_dim: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load().sparstar_workspace_size(int(heads), int(n_q), Segments(n_text, n_ctx, n_cur), int(head_dim),
+                                          ctypes.byref(out)), "sparstar_workspace_size")
+    return int(out.value)
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("q/k/v must be contiguous bf16 CUDA tensors of shape [H, N, d]")
+
+
+class Workspace:
+    """Reusable device workspace sized for one shape (allocated once by torch)."""
+
+    def __init__(self, heads, n_q, n_text, n_ctx, n_cur, head_dim, device):
+        nbytes = workspace_size(heads, n_q, n_text, n_ctx, n_cur, head_dim)
+        self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        self.nbytes = nbytes
+
+
+def select(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_cur: int, clip: int, density: float,
+           budget_mode: int = BUDGET_LITERAL, want_scores: bool = False, workspace: Optional[Workspace] = None,
+           idx: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None, stream=None):
+    """Block selection. Returns (idx [H,nqb,K_total] int32, cnt [H,nqb] int32, scores or None)."""
+    _check_qkv(q, k)
+    H, n_q, d = q.shape
+    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode)
+    nqb, nkb, kmax = int(plan.nqb), int(plan.nkb), max(int(plan.k_total), 1)
+    if idx is None:
+        idx = torch.empty(H, nqb, kmax, dtype=torch.int32, device=q.device)
+    if cnt is None:
+        cnt = torch.empty(H, nqb, dtype=torch.int32, device=q.device)
+    scores = torch.empty(H, nqb, nkb, dtype=torch.float32, device=q.device) if want_scores else None
+    if workspace is None:
+        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device)
+    _check(load().sparstar_select(_ptr(q), _ptr(k), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
+                                  float(density), int(budget_mode), _ptr(idx), _ptr(cnt), idx.shape[-1],
+                                  _ptr(scores), _ptr(workspace.buf), workspace.nbytes, _stream_ptr(stream)),
+           "sparstar_select")
+    return idx, cnt, scores
+
+
+def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor,
+         sm_scale: float = 0.0, o: Optional[torch.Tensor] = None, want_lse: bool = True,
+         lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Block-sparse attention over the kept tiles. Returns (o bf16 [H,Nq,d], lse fp32 [H,Nq] or None)."""
+    _check_qkv(q, k, v)
+    H, n_q, d = q.shape
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous() or not cnt.is_contiguous():
+        raise ValueError("idx/cnt must be contiguous int32")
+    if o is None:
+        o = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty(H, n_q, dtype=torch.float32, device=q.device)
+    _check(load().sparstar_attn(_ptr(q), _ptr(k), _ptr(v), H, n_q, k.shape[1], d, _ptr(idx), _ptr(cnt),
+                                idx.shape[-1], float(sm_scale), _ptr(o), _ptr(lse), _stream_ptr(stream)),
+           "sparstar_attn")
+    return o, lse
+
+
+def forward(q, k, v, n_text, n_ctx, n_cur, clip, density, budget_mode=BUDGET_LITERAL, sm_scale=0.0,
+            workspace: Optional[Workspace] = None, idx=None, cnt=None, o=None, lse=None, want_lse=True,
+            stream=None):
+    """The whole per-scale path (selection then attention). Returns (o, lse, idx, cnt)."""
+    _check_qkv(q, k, v)
+    H, n_q, d = q.shape
+    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode)
+    kmax = max(int(plan.k_total), 1)
+    if idx is None:
+        idx = torch.empty(H, int(plan.nqb), kmax, dtype=torch.int32, device=q.device)
+    if cnt is None:
+        cnt = torch.empty(H, int(plan.nqb), dtype=torch.int32, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty(H, n_q, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device)
+    _check(load().sparstar_forward(_ptr(q), _ptr(k), _ptr(v), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
+                                   float(density), int(budget_mode), float(sm_scale), _ptr(idx), _ptr(cnt),
+                                   idx.shape[-1], _ptr(o), _ptr(lse), _ptr(workspace.buf), workspace.nbytes,
+                                   _stream_ptr(stream)), "sparstar_forward")
+    return o, lse, idx, cnt
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    """Synchronize and return the device status code (OK, ERR_DEVICE_TIMEOUT or ERR_DEVICE_BOUNDS)."""
+    return int(load().sparstar_device_status(_stream_ptr(stream), 1 if clear else 0))
+
+
+def exported_symbols():
+    return list(_SIGNATURES)

@@ -1,0 +1,150 @@
+/*
+ * sparstar.h — C ABI of the B200 (sm_100a) SparSTAR block-sparse attention library.
+ *
+ * The library computes, for one expensive scale of a SpaceTime-AutoRegressive video model,
+ * the training-free dynamic block-sparse attention described in the SparSTAR digest
+ * ("SparSTAR的贡献：每尺度动态重建", pchao.org, section 方法概览 "method overview") and in the
+ * English abstract ("SparSTAR: Sparse Attention for SpaceTime AutoRegressive Video
+ * Synthesis", newx.sg, section Abstract):
+ *   per head, Q and the mixed KV context (text ‖ reference context ‖ current-scale tokens)
+ *   are cut into 128-token blocks; each block is mean-pooled; every (query block, key
+ *   block) pair is scored from the pooled vectors; text blocks (and, in Clip 1, the image
+ *   pyramid blocks) are always kept; the rest of each query-block row is filled by a joint
+ *   Top-K; forward-only attention then runs over the kept blocks only.
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   score      S_ij = mean(q_i) . mean(k_j) / sqrt(d), fp32;
+ *   budget     SPARSTAR_BUDGET_LITERAL: each row holds max(ceil(density * nkb), n_forced)
+ *              blocks; SPARSTAR_BUDGET_CANDIDATES: Top-K adds ceil(density * n_cand)
+ *              blocks to the forced ones;
+ *   ties       equal scores rank the lower block index first; -0.0 equals +0.0;
+ *   ragged     a partial last block is pooled over (and attends to) its valid tokens only;
+ *   blocks     counted over the concatenated KV; a block holding any forced token is forced;
+ *   attention  no causal mask; softmax scale sm_scale (<= 0 selects 1/sqrt(d)).
+ *
+ * Memory layout (all device pointers, row-major, contiguous, 16-byte aligned):
+ *   q   bf16 [H, Nq,  d]      k, v bf16 [H, Nkv, d]      o bf16 [H, Nq, d]
+ *   lse fp32 [H, Nq]          (natural-log sum of exp of the scaled logits; optional)
+ *   idx int32 [H, nqb, kmax]  (kept KV block ids of each row, ascending; only the first
+ *                              cnt entries of a row are written and read)
+ *   cnt int32 [H, nqb]
+ * with nqb = ceil(Nq/128), nkb = ceil(Nkv/128), Nkv = n_text + n_ctx + n_cur.
+ *
+ * Ownership: the caller allocates and owns every buffer; the library allocates no device
+ * memory in these calls. All calls are asynchronous on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and return after enqueuing. Argument errors are detected on
+ * the host before anything is enqueued and leave every output untouched.
+ *
+ * Device-side faults never trap: each kernel bounds its waits and index reads, records a
+ * flag in a per-device status word, and exits. sparstar_device_status() reports it.
+ */
+#ifndef SPARSTAR_H
+#define SPARSTAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARSTAR_BLOCK 128
+#define SPARSTAR_ABI_VERSION 1
+
+/* Return codes. */
+#define SPARSTAR_OK 0
+#define SPARSTAR_ERR_ARG 1             /* bad pointer, size, alignment, density or clip */
+#define SPARSTAR_ERR_UNSUPPORTED 2     /* head_dim not in {64,128}, device not sm_100, size beyond a limit */
+#define SPARSTAR_ERR_WORKSPACE 3       /* workspace NULL or smaller than sparstar_workspace_size() */
+#define SPARSTAR_ERR_CUDA 4            /* a CUDA runtime/driver call failed */
+#define SPARSTAR_ERR_DEVICE_TIMEOUT 5  /* a kernel's bounded wait expired (reported by sparstar_device_status) */
+#define SPARSTAR_ERR_DEVICE_BOUNDS 6   /* a kernel clamped an out-of-range idx/cnt entry */
+
+/* Budget readings (see the header comment). */
+#define SPARSTAR_BUDGET_LITERAL 0
+#define SPARSTAR_BUDGET_CANDIDATES 1
+
+/* KV context = n_text text tokens ‖ n_ctx reference tokens ‖ n_cur current-scale tokens.
+ * In Clip 1 the reference tokens are the image pyramid, in later clips the preceding
+ * clip's final scale (digest, section 这篇论文解决什么问题 and bullet clip感知保留策略). */
+typedef struct sparstar_segments {
+    int64_t n_text;
+    int64_t n_ctx;
+    int64_t n_cur;
+} sparstar_segments;
+
+/* Block counts and per-row budget of one scale. */
+typedef struct sparstar_plan {
+    int64_t nqb;       /* query blocks, ceil(Nq/128) */
+    int64_t nkb;       /* KV blocks, ceil(Nkv/128) */
+    int64_t n_forced;  /* forced (always kept) KV blocks, a prefix 0..n_forced-1 */
+    int64_t n_cand;    /* nkb - n_forced, the blocks Top-K chooses from */
+    int32_t k_total;   /* blocks kept per row (= every row's cnt) */
+    int32_t k_topk;    /* of which chosen by Top-K */
+} sparstar_plan;
+
+/* Host only. Block partition, clip-aware forced prefix and row budget (digest, 方法概览:
+ * 128-token blocks; text, plus Clip-1 pyramid, kept dense; the rest filled by joint Top-K).
+ * clip >= 1; 0 < density <= 1; budget_mode is SPARSTAR_BUDGET_*. n_q may be 0.
+ * Returns SPARSTAR_ERR_ARG on bad input (out untouched). */
+int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double density,
+                       int budget_mode, sparstar_plan* out);
+
+/* Host only. Bytes of device workspace that sparstar_select / sparstar_forward need for
+ * these sizes (pooled block means and, unless the caller passes `scores`, the score
+ * matrix). Writes *bytes; returns SPARSTAR_ERR_ARG on bad sizes. */
+int sparstar_workspace_size(int heads, int64_t n_q, sparstar_segments seg, int head_dim,
+                            size_t* bytes);
+
+/* Block selection (digest, 方法概览: block partition and aggregate scoring, clip-aware
+ * retention, joint Top-K, per-head masks). Reads q [H,Nq,d] and k [H,Nkv,d] (bf16, device),
+ * writes idx [H,nqb,kmax] (first plan.k_total entries of each row, ascending) and
+ * cnt [H,nqb] (= plan.k_total). If `scores` is not NULL it must hold H*nqb*nkb floats and
+ * receives every S_ij (forced columns included); it is then used instead of workspace for
+ * the scores. Rows whose budget is already filled by the forced blocks (k_topk == 0), or
+ * that keep every block, do not depend on the scores: q and k are then not read unless
+ * `scores` was requested.
+ * workspace: device, >= sparstar_workspace_size() bytes, 256-byte aligned.
+ * Requirements: heads >= 1, n_q >= 0, Nkv >= 1, head_dim in {64,128}, kmax >= k_total,
+ * n_cand <= 16384. n_q == 0 is a no-op. */
+int sparstar_select(const void* q, const void* k, int heads, int64_t n_q,
+                    sparstar_segments seg, int head_dim, int clip, double density,
+                    int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
+                    float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward-only block-sparse attention over the kept tiles (digest, 方法概览 bullet
+ * FastFlex执行路径: attention executed over the selected blocks only, with online softmax).
+ * For every valid query token t of query block i of head h:
+ *   o_t = sum over valid KV tokens u of the blocks idx[h][i][0..cnt-1] of
+ *         softmax_u(sm_scale * q_t . k_u) v_u,   lse_t = log sum_u exp(sm_scale * q_t . k_u).
+ * q [H,Nq,d], k/v [H,Nkv,d] bf16 device; o [H,Nq,d] bf16 device (written);
+ * lse fp32 [H,Nq] device or NULL. idx entries must lie in [0,nkb) and cnt in [1,kmax]:
+ * out-of-range entries are clamped and SPARSTAR_ERR_DEVICE_BOUNDS is recorded.
+ * Requires an sm_100 device. n_q == 0 is a no-op. */
+int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_t n_q,
+                  int64_t n_kv, int head_dim, const int32_t* idx, const int32_t* cnt,
+                  int32_t kmax, float sm_scale, void* o, float* lse, void* stream);
+
+/* sparstar_select followed by sparstar_attn on the same stream (the whole per-scale path). */
+int sparstar_forward(const void* q, const void* k, const void* v, int heads, int64_t n_q,
+                     sparstar_segments seg, int head_dim, int clip, double density,
+                     int budget_mode, float sm_scale, int32_t* idx, int32_t* cnt,
+                     int32_t kmax, void* o, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, then returns SPARSTAR_OK, SPARSTAR_ERR_DEVICE_TIMEOUT or
+ * SPARSTAR_ERR_DEVICE_BOUNDS from the current device's status word (timeout wins), or
+ * SPARSTAR_ERR_CUDA if the synchronization itself failed. clear != 0 resets the word. */
+int sparstar_device_status(void* stream, int clear);
+
+/* Static text for a return code (never NULL). */
+const char* sparstar_strerror(int code);
+
+/* SPARSTAR_ABI_VERSION of the loaded library. */
+int sparstar_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSTAR_H */

@@ -1,0 +1,115 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the header
+declares, computes plans and workspace sizes, and rejects bad arguments before touching
+the device (no compute calls are made here)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_attention_tok_b200 import sparstar, _build
+from oracle import sparstar_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sparstar.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_build.LIB_PATH):
+        _build.build()
+    return sparstar.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparstar_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 8
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(sparstar.exported_symbols()) == names
+
+
+def test_abi_version_and_strerror(lib):
+    assert lib.sparstar_abi_version() == 1
+    for code in range(7):
+        assert sparstar.strerror(code)
+    assert sparstar.strerror(99) == "unknown status"
+
+
+@pytest.mark.parametrize("n_q,n_text,n_ctx,n_cur,clip,density", [
+    (1024, 256, 768, 1024, 2, 0.25), (18432, 512, 4096, 18432, 1, 0.1875),
+    (72000, 512, 8192, 72000, 1, 0.09375), (72192, 512, 72192, 72192, 2, 0.09375),
+    (8192, 512, 8192, 8192, 1, 0.625), (5, 200, 300, 1, 1, 0.5), (300, 0, 0, 129, 2, 1.0),
+    (128, 1000, 0, 5, 2, 0.01), (0, 10, 10, 10, 1, 0.3),
+])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_plan_matches_oracle_budget(lib, n_q, n_text, n_ctx, n_cur, clip, density, mode):
+    plan = sparstar.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode)
+    nkb = O.num_blocks(n_text + n_ctx + n_cur)
+    n_forced = min(O.forced_block_count(n_text, n_ctx, clip), nkb)
+    assert plan.nqb == O.num_blocks(n_q) and plan.nkb == nkb
+    assert plan.n_forced == n_forced and plan.n_cand == nkb - n_forced
+    assert (plan.k_total, plan.k_topk) == O.row_budget(nkb, n_forced, density, mode)
+
+
+def test_workspace_size(lib):
+    # pooled q (H*nqb*d), pooled k (H*nkb*d) and scores (H*nqb*nkb), fp32, 256-byte aligned
+    got = sparstar.workspace_size(32, 72192, 512, 72192, 72192, 128)
+    def al(x):
+        return (x + 255) // 256 * 256
+    assert got == al(32 * 564 * 128 * 4) + al(32 * 1132 * 128 * 4) + al(32 * 564 * 1132 * 4)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(density=0.0), sparstar.ERR_ARG), (dict(density=1.5), sparstar.ERR_ARG),
+    (dict(density=float("nan")), sparstar.ERR_ARG), (dict(clip=0), sparstar.ERR_ARG),
+    (dict(mode=7), sparstar.ERR_ARG), (dict(n_text=-1), sparstar.ERR_ARG),
+    (dict(d=96), sparstar.ERR_UNSUPPORTED), (dict(heads=0), sparstar.ERR_ARG),
+    (dict(kmax=1), sparstar.ERR_ARG), (dict(q=0x1008), sparstar.ERR_ARG),
+    (dict(q=None), sparstar.ERR_ARG), (dict(ws=None), sparstar.ERR_WORKSPACE),
+    (dict(ws_bytes=10), sparstar.ERR_WORKSPACE), (dict(ws=0x2010), sparstar.ERR_WORKSPACE),
+])
+def test_select_rejects_bad_arguments_before_launch(lib, kwargs, code):
+    a = dict(q=0x1000, k=0x2000, heads=2, n_q=1024, n_text=256, n_ctx=768, n_cur=1024, d=64, clip=2,
+             density=0.25, mode=0, idx=0x3000, cnt=0x4000, kmax=8, scores=None, ws=0x10000,
+             ws_bytes=1 << 30)
+    a.update(kwargs)
+    rc = lib.sparstar_select(a["q"], a["k"], a["heads"], a["n_q"],
+                             sparstar.Segments(a["n_text"], a["n_ctx"], a["n_cur"]), a["d"], a["clip"],
+                             a["density"], a["mode"], a["idx"], a["cnt"], a["kmax"], a["scores"], a["ws"],
+                             a["ws_bytes"], None)
+    assert rc == code
+
+
+def test_select_zero_queries_is_a_noop(lib):
+    rc = lib.sparstar_select(None, None, 2, 0, sparstar.Segments(256, 768, 1024), 64, 2, 0.25, 0, None, None, 4,
+                             None, None, 0, None)
+    assert rc == sparstar.OK
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(d=80), sparstar.ERR_UNSUPPORTED), (dict(n_kv=0), sparstar.ERR_ARG), (dict(heads=0), sparstar.ERR_ARG),
+    (dict(v=None), sparstar.ERR_ARG), (dict(o=0x5004), sparstar.ERR_ARG), (dict(lse=0x6002), sparstar.ERR_ARG),
+    (dict(kmax=0), sparstar.ERR_ARG), (dict(scale=float("inf")), sparstar.ERR_ARG),
+])
+def test_attn_rejects_bad_arguments_before_launch(lib, kwargs, code):
+    a = dict(q=0x1000, k=0x2000, v=0x3000, heads=2, n_q=1024, n_kv=2048, d=64, idx=0x4000, cnt=0x4800, kmax=4,
+             scale=0.0, o=0x5000, lse=None)
+    a.update(kwargs)
+    rc = lib.sparstar_attn(a["q"], a["k"], a["v"], a["heads"], a["n_q"], a["n_kv"], a["d"], a["idx"], a["cnt"],
+                           a["kmax"], a["scale"], a["o"], a["lse"], None)
+    assert rc == code
+    assert lib.sparstar_attn(None, None, None, 1, 0, 10, 64, None, None, 1, 0.0, None, None, None) == sparstar.OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sparstar, "_LIB", None)
+    monkeypatch.setattr(_build, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        sparstar.load()

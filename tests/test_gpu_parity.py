@@ -1,0 +1,204 @@
+"""CUDA path vs CPU oracle, element by element, through the C ABI.
+
+Small cases are compared on every output; the full-size workloads (launched exactly as
+bench.py launches them) are compared on every mask row and on sampled query blocks of
+the attention output. Inputs are seeded (block_sparse_attention_tok_b200.synth); the
+oracle always reads the exact bytes the GPU used.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_tok_b200 import synth
+from oracle import sparstar_oracle as O
+from tests.parity import bits, check_masks, check_output, LSE_ABS
+
+pytestmark = pytest.mark.gpu
+
+
+def _f64(x_bits):
+    return O.bf16_bits_to_f64(x_bits)
+
+
+def _oracle_attention(qb, kb, vb, rows, h, qblocks, d):
+    qf, kf, vf = _f64(qb[h]), _f64(kb[h]), _f64(vb[h])
+    return O.block_sparse_attention(qf, kf, vf, rows, qblocks)
+
+
+def _run_case(lib, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, qblocks_per_head=None, heads=None):
+    """Forward on the GPU; mask rule on all rows; outputs on rows whose mask equals the oracle's."""
+    S = lib
+    H, n_q, d = q.shape
+    o, lse, idx, cnt = S.forward(q, k, v, n_text, n_ctx, n_cur, clip, density, mode)
+    _, _, scores = S.select(q, k, n_text, n_ctx, n_cur, clip, density, mode, want_scores=True)
+    assert S.device_status() == S.OK
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    ref_idx, ref_S = O.select(qb, kb, n_text, n_ctx, clip, density, mode)
+    plan = S.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode)
+    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    stats = check_masks(gidx, gcnt, ref_idx, ref_S, int(plan.n_forced), int(plan.k_topk))
+    # the fp32 scores the kernel ranked by, against the fp64 definition
+    np.testing.assert_allclose(scores.cpu().numpy(), ref_S, rtol=0, atol=2e-5)
+    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    nqb = int(plan.nqb)
+    for h in (range(H) if heads is None else heads):
+        qbl = range(nqb) if qblocks_per_head is None else qblocks_per_head(nqb)
+        qbl = [i for i in qbl if (gidx[h, i, :ref_idx.shape[2]] == ref_idx[h, i]).all()]
+        outs = _oracle_attention(qb, kb, vb, ref_idx[h], h, qbl, d)
+        for i, (o_ref, lse_ref) in zip(qbl, outs):
+            s, e = O.block_token_range(i, n_q)
+            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
+            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+    return stats
+
+
+def _attn_with_oracle_mask(lib, q, k, v, rows_all, qblocks=None):
+    """sparstar_attn driven by the oracle's own idx rows (uploaded), compared row by row."""
+    S = lib
+    H, n_q, d = q.shape
+    idx = torch.from_numpy(rows_all.astype(np.int32)).to(q.device).contiguous()
+    cnt = torch.full(rows_all.shape[:2], rows_all.shape[2], dtype=torch.int32, device=q.device)
+    o, lse = S.attn(q, k, v, idx, cnt)
+    assert S.device_status() == S.OK
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(H):
+        qbl = list(range(rows_all.shape[1])) if qblocks is None else qblocks
+        for i, (o_ref, lse_ref) in zip(qbl, _oracle_attention(qb, kb, vb, rows_all[h], h, qbl, d)):
+            s, e = O.block_token_range(i, n_q)
+            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
+            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+
+
+@pytest.fixture(scope="module")
+def S(cuda_lib):
+    from block_sparse_attention_tok_b200 import sparstar
+    return sparstar
+
+
+def test_tiny_clip2_scale_all_rows(S):
+    sc = synth.TINY_CLIP2
+    q, k, v = synth.make_scale_inputs(sc, device="cuda")
+    stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, 0)
+    assert stats["identical"] == stats["rows"]
+
+
+@pytest.mark.parametrize("case", list(synth.random_small_cases(seed=4321, count=16)), ids=lambda c: c["name"])
+def test_small_ragged_cases(S, case):
+    c = case
+    q, k, v = synth.make_qkv(c["n_q"], c["n_text"] + c["n_ctx"] + c["n_cur"], c["H"], c["d"],
+                             [c["seed"] + 100 * h for h in range(c["H"])], device="cuda")
+    _run_case(S, q, k, v, c["n_text"], c["n_ctx"], c["n_cur"], c["clip"], c["density"], c["mode"])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n_q,n_kv", [(1, 1), (127, 129), (384, 1000), (700, 3000)])
+def test_attention_on_random_masks(S, d, n_q, n_kv):
+    """Arbitrary ascending kept lists (not only Top-K ones), including a single kept block."""
+    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [7, 8], device="cuda")
+    nqb, nkb = O.num_blocks(n_q), O.num_blocks(n_kv)
+    rng = np.random.default_rng(n_q * 31 + n_kv)
+    kk = max(1, min(nkb, int(rng.integers(1, nkb + 1))))
+    rows = np.stack([np.stack([np.sort(rng.choice(nkb, kk, replace=False)) for _ in range(nqb)])
+                     for _ in range(2)])
+    _attn_with_oracle_mask(S, q, k, v, rows)
+
+
+def test_dense_density_one_matches_oracle(S):
+    q, k, v = synth.make_qkv(640, 1100, 2, 128, [11, 12], device="cuda")
+    stats = _run_case(S, q, k, v, 100, 300, 700, 2, 1.0, 0)
+    assert stats["identical"] == stats["rows"]
+
+
+def test_forced_only_rows(S):
+    # Clip 1 where the text + pyramid prefix fills the budget: K_topk = 0.
+    q, k, v = synth.make_qkv(512, 128 * 12, 2, 128, [21, 22], device="cuda")
+    plan = S.make_plan(512, 256, 768, 512, 1, 0.25)
+    assert plan.k_topk == 0 and plan.k_total == 8
+    stats = _run_case(S, q, k, v, 256, 768, 512, 1, 0.25, 0)
+    assert stats["identical"] == stats["rows"]
+
+
+def test_planted_ties_go_to_lower_index(S):
+    # Duplicate KV blocks have bit-identical pooled means and scores on the GPU as well.
+    H, d = 2, 128
+    q, k, v = synth.make_qkv(256, 128 * 10, H, d, [31, 32], device="cuda")
+    for src, dst in ((3, 7), (4, 8), (5, 9)):
+        k[:, dst * 128:(dst + 1) * 128] = k[:, src * 128:(src + 1) * 128]
+    idx, cnt, sc = S.select(q, k, 128, 0, 128 * 9, 2, 0.5, 0, want_scores=True)
+    ref_idx, _ = O.select(bits(q), bits(k), 128, 0, 2, 0.5, 0)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    s = sc.cpu().numpy()
+    assert np.array_equal(s[:, :, 3], s[:, :, 7]) and np.array_equal(s[:, :, 5], s[:, :, 9])
+
+
+def test_zero_queries_is_noop(S):
+    q = torch.empty(2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(2, 300, 64, dtype=torch.bfloat16, device="cuda")
+    o, lse, idx, cnt = S.forward(q, k, k.clone(), 100, 100, 100, 2, 0.5)
+    assert o.shape == (2, 0, 64) and S.device_status() == S.OK
+
+
+def test_out_of_range_index_is_clamped_and_reported(S):
+    q, k, v = synth.make_qkv(256, 512, 1, 64, [41], device="cuda")
+    idx = torch.tensor([[[0, 1], [2, 99]]], dtype=torch.int32, device="cuda")   # 99 >= nkb = 4
+    cnt = torch.tensor([[2, 2]], dtype=torch.int32, device="cuda")
+    S.device_status(clear=True)
+    S.attn(q, k, v, idx, cnt)
+    assert S.device_status(clear=True) == S.ERR_DEVICE_BOUNDS
+    cnt = torch.tensor([[2, 7]], dtype=torch.int32, device="cuda")             # 7 > kmax = 2
+    idx = torch.tensor([[[0, 1], [2, 3]]], dtype=torch.int32, device="cuda")
+    S.attn(q, k, v, idx, cnt)
+    assert S.device_status(clear=True) == S.ERR_DEVICE_BOUNDS
+    idx = torch.tensor([[[0, 1], [2, 3]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[2, 2]], dtype=torch.int32, device="cuda")
+    S.attn(q, k, v, idx, cnt)
+    assert S.device_status(clear=True) == S.OK
+
+
+def test_custom_softmax_scale(S):
+    q, k, v = synth.make_qkv(300, 700, 1, 128, [51], device="cuda")
+    rows = np.array([[[0, 2, 5], [1, 3, 4], [0, 1, 2]]])
+    idx = torch.from_numpy(rows.astype(np.int32)).cuda()
+    cnt = torch.full((1, 3), 3, dtype=torch.int32, device="cuda")
+    o, lse = S.attn(q, k, v, idx, cnt, sm_scale=0.05)
+    qf, kf, vf = (_f64(bits(x)[0]) for x in (q, k, v))
+    outs = O.block_sparse_attention(qf, kf, vf, rows[0], [0, 1, 2], sm_scale=0.05)
+    o_np = o.float().cpu().numpy()[0]
+    for i, (o_ref, _) in enumerate(outs):
+        s, e = O.block_token_range(i, 300)
+        check_output(o_np[s:e], o_ref, f"qb{i}")
+
+
+def _sampled(nqb):
+    rng = np.random.default_rng(nqb)
+    return sorted({0, nqb - 1, *rng.choice(nqb, 3, replace=False).tolist()})
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", [synth.MID_CLIP1.name, synth.FINAL_CLIP1_RAGGED.name, synth.FINAL_CLIP2.name])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_full_size_scales(S, name, mode):
+    sc = synth.WORKLOADS[name]
+    if mode == 1 and sc.clip == 2:
+        pytest.skip("the candidates budget differs from the literal one only where forced blocks fill the row")
+    q, k, v = synth.make_scale_inputs(sc, device="cuda")
+    stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode,
+                      qblocks_per_head=_sampled, heads=[0, sc.heads - 1])
+    print(name, mode, stats)
+    del q, k, v
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("scale_index", [0, 3])
+@pytest.mark.parametrize("layer", [0, 35])
+def test_schedule_scales(S, scale_index, layer):
+    sc = synth.SCHEDULE_CLIP1[scale_index]
+    q, k, v = synth.make_scale_inputs(sc, device="cuda", layer=layer, scale_index=scale_index)
+    _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, 0,
+              qblocks_per_head=_sampled, heads=[0, 31])
+    del q, k, v
+    torch.cuda.empty_cache()
