@@ -1,0 +1,388 @@
+"""Benchmark of one expensive SparSTAR scale on B200: selection + block-sparse attention.
+
+A step is the whole per-scale path (pooling, scores, Top-K, attention over the kept tiles)
+over one 720p final-scale Clip-2 input (32 heads, d 128, 72,192 query tokens, KV 512 text +
+72,192 preceding-clip + 72,192 current tokens, density 0.09375), inputs resident in HBM.
+
+Prints one JSON line (rank 0). Timed region: barrier + synchronize, K steps bracketed by
+CUDA events on the launch stream, synchronize + barrier; the max over ranks is reported.
+Inputs (3.5 GB per GPU) are far larger than L2 (126 MB), so no flush is inserted.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_attention_tok_b200 import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "sparse-attn TFLOP/s on kept tiles & % of bf16 peak; select GB/s; µs per scale"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=synth.FINAL_CLIP2.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--budget-mode", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every 20 ms (reads only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: no clock record
+            self._nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def kept_tile_flops(idx: torch.Tensor, cnt: torch.Tensor, n_q: int, n_kv: int, d: int) -> float:
+    """4 d * sum over kept tiles of valid_query_rows * valid_kv_tokens (bookkeeping only)."""
+    H, nqb, kmax = idx.shape
+    col = torch.arange(kmax, device=idx.device)
+    live = col[None, None, :] < cnt[:, :, None]
+    nkb = -(-n_kv // 128)
+    vk = torch.where(idx == nkb - 1, n_kv - (nkb - 1) * 128, 128).to(torch.float64)
+    per_row = (vk * live).sum(-1)
+    vq = torch.full((nqb,), 128.0, dtype=torch.float64, device=idx.device)
+    vq[-1] = n_q - (nqb - 1) * 128
+    return float(4.0 * d * (per_row * vq[None, :]).sum().item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(q, k, v, sc, heads, q_sample, budget_mode):
+    """The oracle's whole path on a bounded sample: for each listed head, widen its bf16
+    inputs, run its full selection, and run attention for q_sample evenly spaced query
+    blocks. Returns (kept-tile FLOPs of the sampled blocks, seconds, prorated seconds)."""
+    from oracle import sparstar_oracle as O
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    flops, t_total, t_pro = 0.0, 0.0, 0.0
+    nqb = O.num_blocks(sc.n_q)
+    pick = np.unique(np.linspace(0, nqb - 1, min(q_sample, nqb)).round().astype(int))
+    for h in heads:
+        qh, kh, vh = (x[h].cpu() for x in (q, k, v))
+        t0 = time.perf_counter()
+        qf, kf, vf = (O.bf16_bits_to_f64(bits(x)) for x in (qh, kh, vh))
+        rows, _ = O.select_head(qf, kf, sc.n_text, sc.n_ctx, sc.clip, sc.density, budget_mode)
+        t1 = time.perf_counter()
+        O.block_sparse_attention(qf, kf, vf, rows, pick)
+        t2 = time.perf_counter()
+        for i in pick:
+            s, e = O.block_token_range(int(i), sc.n_q)
+            vk = sum(b - a for a, b in (O.block_token_range(int(j), sc.n_kv) for j in rows[i]))
+            flops += 4.0 * sc.head_dim * (e - s) * vk
+        t_total += t2 - t0
+        t_pro += (t1 - t0) * len(pick) / nqb + (t2 - t1)
+    return flops, t_total, t_pro
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, rank):
+    """--impl reference: the CPU oracle, as it stands, on a bounded sample per step."""
+    if rank != 0:
+        return 0
+    sc = synth.WORKLOADS[args.workload]
+    q_sample = 48
+    heads_total = sc.heads
+    vals, times = [], []
+    for step in range(args.warmup + args.steps):
+        h = step % heads_total
+        seed = 1000 * synth.CFG_INDEX.get(sc.name, 0) + h
+        q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, 1, sc.head_dim, [seed], device="cpu")
+        flops, t, t_pro = oracle_sample(q, k, v, sc, [0], q_sample, args.budget_mode)
+        if step >= args.warmup:
+            vals.append(flops / t_pro / 1e12)
+            times.append(t)
+        del q, k, v
+    value = float(np.mean(vals))
+    cores = _blas_threads()
+    sample = (f"per step one head (cycling 0..{heads_total - 1}): bf16 widening + full selection of that head "
+              f"(prorated to the sampled rows) + attention of {q_sample} evenly spaced query blocks; fp64 numpy")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": float(np.mean(times) * 1e3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(sc, args), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(sc, args):
+    return {"workload": sc.name, "heads": sc.heads, "head_dim": sc.head_dim, "n_q": sc.n_q,
+            "kv": {"text": sc.n_text, "ctx": sc.n_ctx, "cur": sc.n_cur}, "clip": sc.clip,
+            "density": sc.density, "budget": "literal" if args.budget_mode == 0 else "candidates",
+            "block": 128, "per_gpu": "one full scale (all heads) per rank",
+            "l2": "no flush: inputs 3.5 GB per GPU > 126 MB L2", "parallelism": f"replicas x{args.gpus}"}
+
+
+def run_ours(args, rank, world, local_rank):
+    from block_sparse_attention_tok_b200 import sparstar as S
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    S.load()
+    sc = synth.WORKLOADS[args.workload]
+    seeds = [1000 * synth.CFG_INDEX.get(sc.name, 0) + h + 100000 * rank for h in range(sc.heads)]
+    q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim, seeds, device=dev)
+    plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode)
+    kmax = int(plan.k_total)
+    ws = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
+    idx = torch.empty(sc.heads, int(plan.nqb), kmax, dtype=torch.int32, device=dev)
+    cnt = torch.empty(sc.heads, int(plan.nqb), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(sc.heads, sc.n_q, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    seg = (sc.n_text, sc.n_ctx, sc.n_cur)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        S.select(q, k, *seg, sc.clip, sc.density, args.budget_mode, workspace=ws, idx=idx, cnt=cnt)
+        if ev is not None:
+            ev[1].record(stream)
+        S.attn(q, k, v, idx, cnt, o=o, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            t = torch.zeros(1, device=dev)
+            dist.all_reduce(t)
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    assert S.device_status() == S.OK
+    flops = kept_tile_flops(idx, cnt, sc.n_q, sc.n_kv, sc.head_dim)
+    launches_per_step = (3 if 0 < plan.k_topk < plan.n_cand else 1) + 1
+    sel_bytes = 2.0 * sc.heads * sc.head_dim * (sc.n_q + sc.n_kv) + 4.0 * sc.heads * plan.nqb * (kmax + 1)
+    if plan.k_topk == 0 or plan.k_topk == plan.n_cand:
+        sel_bytes = 4.0 * sc.heads * plan.nqb * (kmax + 1)   # rows do not depend on the inputs
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    t_sel = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    status = S.device_status()
+    if world > 1:
+        t = torch.tensor([ms, t_sel, t_att], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, t_sel, t_att = (float(x) for x in t.tolist())
+
+    peaks, peak_src = load_peaks()
+    attn_tflops = flops / (t_att * 1e-3) / 1e12
+    sel_gbs = sel_bytes / (t_sel * 1e-3) / 1e9
+    peak_t = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak_hbm = float(peaks["hbm_gbs"])
+    result = {
+        "metric": METRIC,
+        "value": world * flops / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(sc, args),
+        "gpu_launches": launches_per_step * args.steps,
+        "attn": {"ms": t_att, "tflops": attn_tflops, "frac_of_peak": attn_tflops / peak_t,
+                 "kept_tile_tflop": flops / 1e12, "kept_blocks_per_row": kmax},
+        "select": {"us": t_sel * 1e3, "gbs": sel_gbs, "frac_of_hbm": sel_gbs / peak_hbm,
+                   "bytes": sel_bytes, "share_of_step": t_sel / (t_sel + t_att)},
+        "us_per_scale": ms * 1e3,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak_t, "traffic": None,
+                     "kernel": "attn_sparse_kernel<128>",
+                     "peak_source": f"{peak_src} bf16 sustained (kernel inside a back-to-back step loop)"},
+        "device_status": int(status),
+    }
+    clocks_summary = clocks.summary()
+    result["clocks"] = clocks_summary
+
+    # dense run of the same shape: the same kernel with every block kept
+    if not args.no_dense:
+        dplan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, 1.0)
+        didx = torch.arange(int(dplan.nkb), dtype=torch.int32, device=dev).expand(
+            sc.heads, int(dplan.nqb), int(dplan.nkb)).contiguous()
+        dcnt = torch.full((sc.heads, int(dplan.nqb)), int(dplan.nkb), dtype=torch.int32, device=dev)
+        S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1)
+        dflops = kept_tile_flops(didx, dcnt, sc.n_q, sc.n_kv, sc.head_dim)
+        result["dense"] = {"ms": dms, "tflops": dflops / (dms * 1e-3) / 1e12,
+                           "speedup_of_sparse_step": dms / ms}
+        del didx, dcnt
+
+    # end to end through the public API with host buffers: H2D of q/k/v, forward, D2H of o
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        n_e2e = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            S.forward(q, k, v, *seg, sc.clip, sc.density, args.budget_mode, workspace=ws, idx=idx, cnt=cnt,
+                      o=o, lse=lse)
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        result["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+                         "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+                         "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e}
+        del hq, hk, hv, ho
+
+    if rank == 0 and not args.no_cpu_baseline:
+        qc, kc, vc = (x[:2].cpu() for x in (q, k, v))
+        fl, t, t_pro = oracle_sample(qc, kc, vc, sc, [0, 1], 96, args.budget_mode)
+        result["cpu_baseline"] = {
+            "value": fl / t_pro / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": "heads 0-1 of the same input: bf16 widening + full selection (prorated to the sampled "
+                      "rows) + attention of 96 evenly spaced query blocks per head, fp64 numpy; "
+                      f"{t:.1f} s of CPU time"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

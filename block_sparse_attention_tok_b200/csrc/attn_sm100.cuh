@@ -336,7 +336,8 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         seq.n = n;
         const int j = seq_block(seq, p, false);
         const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * 128) : 128;
-        if (!mbar_wait(&s_full[s], tiles & 1u, abort_flag, p.status)) {
+        // tcgen05.ld/st below are warp-collective: every lane must take the same path.
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], tiles & 1u, abort_flag, p.status))) {
           ok = false;
           break;
         }
@@ -360,13 +361,14 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
           for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[c][e]));
         const float mx_scaled = mx * p.scale_log2;
         float alpha = 1.f;
-        bool rescale = false;
         if (mx_scaled > m_run + 8.f) {
           alpha = ex2_approx(m_run - mx_scaled);  // m_run = -inf on the first tile -> 0
           l_run *= alpha;
           m_run = mx_scaled;
-          rescale = (n > 0);
         }
+        // O is rescaled by the whole warp when any of its rows moved its max (alpha = 1
+        // leaves the other rows unchanged); the first tile overwrites O instead.
+        const bool rescale = n > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f);
         float rowsum = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> bf16, lse
-      if (!mbar_wait(&o_full[s], items & 1u, abort_flag, p.status)) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_full[s], items & 1u, abort_flag, p.status))) break;
       ++items;
       tc_fence_after();
       const int64_t t = static_cast<int64_t>(seq.qb) * 128 + row;

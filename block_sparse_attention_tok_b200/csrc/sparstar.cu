@@ -296,7 +296,6 @@ int sparstar_forward(const void* q, const void* k, const void* v, int heads, int
                      int head_dim, int clip, double density, int budget_mode, float sm_scale, int32_t* idx,
                      int32_t* cnt, int32_t kmax, void* o, float* lse, void* workspace, size_t workspace_bytes,
                      void* stream) {
-  if (v == nullptr || o == nullptr) return SPARSTAR_ERR_ARG;
   int rc = sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
                            workspace, workspace_bytes, stream);
   if (rc != SPARSTAR_OK) return rc;

@@ -28,29 +28,34 @@ def _oracle_attention(qb, kb, vb, rows, h, qblocks, d):
 
 
 def _run_case(lib, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, qblocks_per_head=None, heads=None):
-    """Forward on the GPU; mask rule on all rows; outputs on rows whose mask equals the oracle's."""
+    """Forward on the GPU; the mask rule on every row of the checked heads; outputs on the
+    query blocks (all, or qblocks_per_head(nqb)) whose mask equals the oracle's."""
     S = lib
     H, n_q, d = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
     o, lse, idx, cnt = S.forward(q, k, v, n_text, n_ctx, n_cur, clip, density, mode)
     _, _, scores = S.select(q, k, n_text, n_ctx, n_cur, clip, density, mode, want_scores=True)
     assert S.device_status() == S.OK
-    qb, kb, vb = bits(q), bits(k), bits(v)
-    ref_idx, ref_S = O.select(qb, kb, n_text, n_ctx, clip, density, mode)
     plan = S.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode)
-    gidx, gcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    sel = torch.tensor(heads, device=q.device)
+    qb, kb, vb = bits(q[sel]), bits(k[sel]), bits(v[sel])
+    ref = [O.select_head(_f64(qb[i]), _f64(kb[i]), n_text, n_ctx, clip, density, mode) for i in range(len(heads))]
+    ref_idx = np.stack([r[0] for r in ref])
+    ref_S = np.stack([r[1] for r in ref])
+    gidx, gcnt = idx[sel].cpu().numpy(), cnt[sel].cpu().numpy()
     stats = check_masks(gidx, gcnt, ref_idx, ref_S, int(plan.n_forced), int(plan.k_topk))
     # the fp32 scores the kernel ranked by, against the fp64 definition
-    np.testing.assert_allclose(scores.cpu().numpy(), ref_S, rtol=0, atol=2e-5)
-    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    np.testing.assert_allclose(scores[sel].cpu().numpy(), ref_S, rtol=0, atol=2e-5)
+    o_np, lse_np = o[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
     nqb = int(plan.nqb)
-    for h in (range(H) if heads is None else heads):
+    for hi in range(len(heads)):
         qbl = range(nqb) if qblocks_per_head is None else qblocks_per_head(nqb)
-        qbl = [i for i in qbl if (gidx[h, i, :ref_idx.shape[2]] == ref_idx[h, i]).all()]
-        outs = _oracle_attention(qb, kb, vb, ref_idx[h], h, qbl, d)
+        qbl = [i for i in qbl if (gidx[hi, i, :ref_idx.shape[2]] == ref_idx[hi, i]).all()]
+        outs = _oracle_attention(qb, kb, vb, ref_idx[hi], hi, qbl, d)
         for i, (o_ref, lse_ref) in zip(qbl, outs):
             s, e = O.block_token_range(i, n_q)
-            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
-            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+            check_output(o_np[hi, s:e], o_ref, f"h{heads[hi]} qb{i}")
+            assert np.abs(lse_np[hi, s:e] - lse_ref).max() <= LSE_ABS
     return stats
 
 
@@ -104,6 +109,29 @@ def test_attention_on_random_masks(S, d, n_q, n_kv):
     rows = np.stack([np.stack([np.sort(rng.choice(nkb, kk, replace=False)) for _ in range(nqb)])
                      for _ in range(2)])
     _attn_with_oracle_mask(S, q, k, v, rows)
+
+
+def test_many_items_per_slot(S):
+    """More (head, query block) items than two per CTA slot: exercises the per-slot item
+    sequence (Q buffer reuse, O handover between items) of the persistent kernel."""
+    q, k, v = synth.make_qkv(128 * 90 + 37, 1100, 8, 128, [61 + h for h in range(8)], device="cuda")
+    stats = _run_case(S, q, k, v, 128, 256, 716, 2, 0.5, 0, qblocks_per_head=lambda n: range(0, n, 7))
+    assert stats["rows"] == 8 * 91
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_row_max_jump_in_some_rows_only(S, d):
+    """Rows 0-15 of every query block meet a much larger logit in a late KV block, so their
+    running max moves (O rescale) while the other rows of the same warp keep theirs."""
+    n_q, n_kv = 128 * 6, 128 * 8
+    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [71, 72], device="cuda")
+    qv = q.view(2, 6, 128, d)
+    qv[:, :, :16, 0] = 16.0
+    k[:, 6 * 128:7 * 128, 0] = 16.0
+    rows = np.tile(np.array([0, 2, 3, 6]), (2, 6, 1))
+    _attn_with_oracle_mask(S, q, k, v, rows)
+    # and the same through the full path with every block kept
+    _run_case(S, q, k, v, 0, 0, n_kv, 2, 1.0, 0)
 
 
 def test_dense_density_one_matches_oracle(S):
@@ -186,7 +214,7 @@ def test_full_size_scales(S, name, mode):
         pytest.skip("the candidates budget differs from the literal one only where forced blocks fill the row")
     q, k, v = synth.make_scale_inputs(sc, device="cuda")
     stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode,
-                      qblocks_per_head=_sampled, heads=[0, sc.heads - 1])
+                      qblocks_per_head=_sampled, heads=[0, 1, sc.heads // 2, sc.heads - 1])
     print(name, mode, stats)
     del q, k, v
     torch.cuda.empty_cache()
