@@ -303,6 +303,41 @@ int sparstar_forward(const void* q, const void* k, const void* v, int heads, int
   return sparstar_attn(q, k, v, heads, n_q, n_kv, head_dim, idx, cnt, kmax, sm_scale, o, lse, stream);
 }
 
+// ---------------------------------------------------------------- no-allocation selection
+// Scratch of sparstar_select_noalloc: a fixed device array per device that loads the library.
+// Host code must not pass `g_select_scratch` itself to a kernel (on the host it names a
+// host-side stand-in); it passes the device address looked up once per device below.
+static __device__ __align__(256) unsigned char g_select_scratch[SPARSTAR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[sparstar::kMaxDevices] = {};
+}  // namespace
+
+int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q, sparstar_segments seg,
+                            int head_dim, int clip, double density, int budget_mode, int32_t* idx, int32_t* cnt,
+                            int32_t kmax, void* stream) {
+  // Sizes are checked before any CUDA call, so an oversized request never touches the device.
+  size_t need = 0;
+  int rc = sparstar_workspace_size(heads, n_q, seg, head_dim, &need);
+  if (rc != SPARSTAR_OK) return rc;
+  if (need > SPARSTAR_NOALLOC_SCRATCH_BYTES) return SPARSTAR_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sparstar::kMaxDevices) return SPARSTAR_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || ptr == nullptr) return SPARSTAR_ERR_CUDA;
+      g_scratch_ptr[dev] = ptr;
+    }
+    scratch = g_scratch_ptr[dev];
+  }
+  return sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
+                         scratch, SPARSTAR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 int sparstar_device_status(void* stream, int clear) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);

@@ -58,7 +58,11 @@ _SIGNATURES.update({
                                     _c.c_int, _c.c_double, _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p,
                                     _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "sparstar_device_status": (_c.c_int, [_c.c_void_p, _c.c_int]),
+    "sparstar_select_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments, _c.c_int,
+                                           _c.c_int, _c.c_double, _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32,
+                                           _c.c_void_p]),
 })
+NOALLOC_SCRATCH_BYTES = 128 << 20
 
 _LIB: Optional[ctypes.CDLL] = None
 
@@ -202,6 +206,26 @@ def forward(q, k, v, n_text, n_ctx, n_cur, clip, density, budget_mode=BUDGET_LIT
                                    idx.shape[-1], _ptr(o), _ptr(lse), _ptr(workspace.buf), workspace.nbytes,
                                    _stream_ptr(stream)), "sparstar_forward")
     return o, lse, idx, cnt
+
+
+def select_noalloc(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_cur: int, clip: int,
+                   density: float, budget_mode: int = BUDGET_LITERAL, idx: Optional[torch.Tensor] = None,
+                   cnt: Optional[torch.Tensor] = None, stream=None):
+    """Block selection without any device allocation inside the library: its scratch is the
+    library's fixed array (NOALLOC_SCRATCH_BYTES per device). For callers that cannot call
+    cudaMalloc; they pass idx and cnt buffers they already own. Calls that overlap on the
+    GPU share that array and race. Returns (idx, cnt)."""
+    _check_qkv(q, k)
+    H, n_q, d = q.shape
+    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode)
+    if idx is None:
+        idx = torch.empty(H, int(plan.nqb), max(int(plan.k_total), 1), dtype=torch.int32, device=q.device)
+    if cnt is None:
+        cnt = torch.empty(H, int(plan.nqb), dtype=torch.int32, device=q.device)
+    _check(load().sparstar_select_noalloc(_ptr(q), _ptr(k), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
+                                          float(density), int(budget_mode), _ptr(idx), _ptr(cnt), idx.shape[-1],
+                                          _stream_ptr(stream)), "sparstar_select_noalloc")
+    return idx, cnt
 
 
 def device_status(clear: bool = True, stream=None) -> int:

@@ -132,6 +132,30 @@ int sparstar_forward(const void* q, const void* k, const void* v, int heads, int
                      int32_t kmax, void* o, float* lse, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* Block selection for callers that cannot allocate device memory: the same computation
+ * and outputs as sparstar_select (with scores == NULL), but the scratch it needs (pooled
+ * block means and the score matrix) lives in a fixed array inside the library instead of
+ * a caller-provided workspace. The paper has no counterpart; this exists for callers that
+ * run where cudaMalloc is unavailable or forbidden, e.g. inside a host framework that owns
+ * all device memory through its own pool, a plugin that must not allocate, or code that
+ * runs while a memory-capping policy is in force.
+ * The array holds SPARSTAR_NOALLOC_SCRATCH_BYTES bytes on every device that loads the
+ * library, until the process exits. Sizes whose sparstar_workspace_size() exceeds it are
+ * rejected with SPARSTAR_ERR_UNSUPPORTED before anything is enqueued.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the last call's contents; every
+ * value a call reads from it is written earlier by the same call, so nothing needs
+ * clearing. Calls whose kernels overlap on the GPU (different streams without ordering,
+ * or several host threads) race on the array: serialize them.
+ * No cudaMalloc, cudaFree or allocating library routine is called. Other arguments,
+ * requirements and return codes are those of sparstar_select. */
+#define SPARSTAR_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
+int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q,
+                            sparstar_segments seg, int head_dim, int clip, double density,
+                            int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
+                            void* stream);
+
 /* Synchronizes `stream`, then returns SPARSTAR_OK, SPARSTAR_ERR_DEVICE_TIMEOUT or
  * SPARSTAR_ERR_DEVICE_BOUNDS from the current device's status word (timeout wins), or
  * SPARSTAR_ERR_CUDA if the synchronization itself failed. clear != 0 resets the word. */
