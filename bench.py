@@ -13,6 +13,7 @@ Inputs (3.5 GB per GPU) are far larger than L2 (126 MB), so no flush is inserted
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -42,6 +43,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=synth.FINAL_CLIP2.name, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget-mode", type=int, default=0)
+    ap.add_argument("--heads", type=int, default=0, help="limit the heads (profiling small cases); 0 = all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -217,6 +219,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     S.load()
     sc = synth.WORKLOADS[args.workload]
+    if args.heads:
+        sc = dataclasses.replace(sc, heads=args.heads)
     seeds = [1000 * synth.CFG_INDEX.get(sc.name, 0) + h + 100000 * rank for h in range(sc.heads)]
     q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim, seeds, device=dev)
     plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode)
