@@ -123,11 +123,56 @@ __device__ __forceinline__ int seq_block(const SlotSeq& s, const AttnParams& p, 
   return clamp_block(j, p.nkb, p.status, report);
 }
 
-template <int D>
+// ------------------------------------------------------------------------ softmax helpers
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Max of a 128-column S row held as four 32-register chunks: 8 independent 3-input max
+// chains, then a short tree (dependency depth 10 instead of 128).
+__device__ __forceinline__ float row_max128(const uint32_t (&r)[4][32]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    m[i] = fmax3(__uint_as_float(r[0][i]), __uint_as_float(r[0][i + 8]), __uint_as_float(r[0][i + 16]));
+#pragma unroll
+  for (int k = 24; k < 128; k += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      m[i] = fmax3(m[i], __uint_as_float(r[(k + i) >> 5][(k + i) & 31]),
+                   __uint_as_float(r[(k + 8 + i) >> 5][(k + 8 + i) & 31]));
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// 2^x on the FMA pipe for a pair of arguments x <= 8: n = round(x) with the 1.5*2^23
+// shifter, f = x - n in [-1/2, 1/2], 2^f by a degree-3 polynomial (coefficients from
+// exp2_poly_fit.py: Chebyshev-node least squares of the relative error, max 1.2e-4), and
+// 2^n added into the exponent field. Arguments below -125 are clamped there (2^-125 is
+// far below anything a bf16 P or the fp32 row sum can register).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c1 = 0.6933686137199402f, c2 = 0.24221783876419067f, c3 = 0.05459282547235489f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+template <int D, int kPolyCols>
 __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
     attn_sparse_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnConfig<D>;
+  static_assert(kPolyCols % 32 == 0 && kPolyCols <= 128, "software exp2 works on whole 32-column chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -183,25 +228,25 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
   if (warp == C::kLoadWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      SlotSeq seq[2];
-      seq_init(seq[0], blockIdx.x * 2 + 0, p, true);
-      seq_init(seq[1], blockIdx.x * 2 + 1, p, true);
+      SlotSeq seq0, seq1;
+      seq_init(seq0, blockIdx.x * 2 + 0, p, true);
+      seq_init(seq1, blockIdx.x * 2 + 1, p, true);
       uint32_t ring_it = 0;
-      int last_q_k[2] = {-1, -1};
+      int last_q_k0 = -1, last_q_k1 = -1;
       bool ok = true;
 
-      auto load_q = [&](int s) -> bool {
-        if (!mbar_wait(&q_empty[s], (seq[s].k & 1) ^ 1, abort_flag, p.status)) return false;
+      auto load_q = [&](int s, SlotSeq& sq, int& last_k) -> bool {
+        if (!mbar_wait(&q_empty[s], (sq.k & 1) ^ 1, abort_flag, p.status)) return false;
         mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
         const uint32_t dst = smem_u32(q_tile + s * C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kChunkBytes, &tm_q, &q_full[s], c * 64, seq[s].qb * 128, seq[s].h);
-        last_q_k[s] = seq[s].k;
+          tma_load_3d(dst + c * C::kChunkBytes, &tm_q, &q_full[s], c * 64, sq.qb * 128, sq.h);
+        last_k = sq.k;
         return true;
       };
-      auto load_kv = [&](int s, const CUtensorMap* map) -> bool {
-        const int j = seq_block(seq[s], p, true);
+      auto load_kv = [&](SlotSeq& sq, const CUtensorMap* map) -> bool {
+        const int j = seq_block(sq, p, true);
         const uint32_t stage = ring_it % C::kStages;
         const uint32_t phase = (ring_it / C::kStages) & 1u;
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
@@ -209,23 +254,26 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         const uint32_t dst = smem_u32(ring + stage * C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kChunkBytes, map, &full[stage], c * 64, j * 128, seq[s].h);
+          tma_load_3d(dst + c * C::kChunkBytes, map, &full[stage], c * 64, j * 128, sq.h);
         ++ring_it;
         return true;
       };
+      // One step of a slot: V of its current tile, then Q (new item) and K of its next tile.
+      auto step = [&](int s, SlotSeq& sq, int& last_k) {
+        if (!ok || sq.item < 0) return;
+        ok = load_kv(sq, &tm_v);
+        if (!ok) return;
+        const bool new_item = seq_next(sq, stride, p, true);
+        if (sq.item < 0) return;
+        if (new_item) ok = load_q(s, sq, last_k);
+        if (ok) ok = load_kv(sq, &tm_k);
+      };
 
-      for (int s = 0; s < 2 && ok; ++s)
-        if (seq[s].item >= 0) ok = load_q(s) && load_kv(s, &tm_k);
-      while (ok && (seq[0].item >= 0 || seq[1].item >= 0)) {
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (seq[s].item < 0) continue;
-          ok = load_kv(s, &tm_v);
-          if (!ok) break;
-          const bool new_item = seq_next(seq[s], stride, p, true);
-          if (seq[s].item < 0) continue;
-          if (new_item) ok = load_q(s);
-          if (ok) ok = load_kv(s, &tm_k);
-        }
+      if (seq0.item >= 0) ok = load_q(0, seq0, last_q_k0) && load_kv(seq0, &tm_k);
+      if (ok && seq1.item >= 0) ok = load_q(1, seq1, last_q_k1) && load_kv(seq1, &tm_k);
+      while (ok && (seq0.item >= 0 || seq1.item >= 0)) {
+        step(0, seq0, last_q_k0);
+        step(1, seq1, last_q_k1);
       }
       // Drain: wait until every load issued into a stage or Q buffer has landed, so no TMA
       // write is in flight when the CTA exits (matters only after an abort).
@@ -237,27 +285,28 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
           }
         }
       }
-      for (int s = 0; s < 2; ++s) {
-        if (last_q_k[s] >= 0) {
-          const unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&q_full[s], last_q_k[s] & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+      auto drain_q = [&](int s, int last_k) {
+        if (last_k < 0) return;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&q_full[s], last_k & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
-      }
+      };
+      drain_q(0, last_q_k0);
+      drain_q(1, last_q_k1);
     }
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      SlotSeq seq[2];
-      seq_init(seq[0], blockIdx.x * 2 + 0, p, false);
-      seq_init(seq[1], blockIdx.x * 2 + 1, p, false);
+      SlotSeq seq0, seq1;
+      seq_init(seq0, blockIdx.x * 2 + 0, p, false);
+      seq_init(seq1, blockIdx.x * 2 + 1, p, false);
       uint32_t ring_it = 0;
-      uint32_t tiles[2] = {0u, 0u};
+      uint32_t tiles0 = 0u, tiles1 = 0u;
       bool ok = true;
 
-      auto issue_s = [&](int s) -> bool {
-        if (seq[s].n == 0 && !mbar_wait(&q_full[s], seq[s].k & 1, abort_flag, p.status)) return false;
+      auto issue_s = [&](int s, const SlotSeq& sq) -> bool {
+        if (sq.n == 0 && !mbar_wait(&q_full[s], sq.k & 1, abort_flag, p.status)) return false;
         const uint32_t stage = ring_it % C::kStages;
         if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
         tc_fence_after();
@@ -272,13 +321,13 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         }
         mma_commit(&empty[stage]);
         mma_commit(&s_full[s]);
-        if (seq[s].n == seq[s].ntiles - 1) mma_commit(&q_empty[s]);
+        if (sq.n == sq.ntiles - 1) mma_commit(&q_empty[s]);
         ++ring_it;
         return true;
       };
-      auto issue_pv = [&](int s) -> bool {
-        if (!mbar_wait(&p_full[s], tiles[s] & 1u, abort_flag, p.status)) return false;
-        ++tiles[s];
+      auto issue_pv = [&](int s, const SlotSeq& sq, uint32_t& tiles) -> bool {
+        if (!mbar_wait(&p_full[s], tiles & 1u, abort_flag, p.status)) return false;
+        ++tiles;
         const uint32_t stage = ring_it % C::kStages;
         if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
         tc_fence_after();
@@ -291,25 +340,28 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
           // V tile is MN-major for this MMA: 64-element chunks of d at 16 KB (LBO), 8-row
           // groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
           mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
-                 (seq[s].n > 0 || kk > 0) ? 1u : 0u);
+                 (sq.n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
-        if (seq[s].n == seq[s].ntiles - 1) mma_commit(&o_full[s]);
+        if (sq.n == sq.ntiles - 1) mma_commit(&o_full[s]);
         ++ring_it;
         return true;
       };
+      // One step of a slot: O += P V for its current tile, then S of its next tile.
+      auto step = [&](int s, SlotSeq& sq, uint32_t& tiles) {
+        if (!ok || sq.item < 0) return;
+        ok = issue_pv(s, sq, tiles);
+        if (!ok) return;
+        seq_next(sq, stride, p, false);
+        if (sq.item < 0) return;
+        ok = issue_s(s, sq);
+      };
 
-      for (int s = 0; s < 2 && ok; ++s)
-        if (seq[s].item >= 0) ok = issue_s(s);
-      while (ok && (seq[0].item >= 0 || seq[1].item >= 0)) {
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (seq[s].item < 0) continue;
-          ok = issue_pv(s);
-          if (!ok) break;
-          seq_next(seq[s], stride, p, false);
-          if (seq[s].item < 0) continue;
-          ok = issue_s(s);
-        }
+      if (seq0.item >= 0) ok = issue_s(0, seq0);
+      if (ok && seq1.item >= 0) ok = issue_s(1, seq1);
+      while (ok && (seq0.item >= 0 || seq1.item >= 0)) {
+        step(0, seq0, tiles0);
+        step(1, seq1, tiles1);
       }
       // Drain: all issued MMAs complete before TMEM is released.
       mma_commit(drain);
@@ -326,6 +378,7 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem_base + lane_off + C::kTmemS + 128u * s;
     const uint32_t t_o = tmem_base + lane_off + C::kTmemO + 128u * s;
+    const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     SlotSeq seq;
     seq_init(seq, blockIdx.x * 2 + s, p, false);
     uint32_t tiles = 0, items = 0;
@@ -354,12 +407,7 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (32 * c + e >= n_valid) r[c][e] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[c][e]));
-        const float mx_scaled = mx * p.scale_log2;
+        const float mx_scaled = row_max128(r) * p.scale_log2;
         float alpha = 1.f;
         if (mx_scaled > m_run + 8.f) {
           alpha = ex2_approx(m_run - mx_scaled);  // m_run = -inf on the first tile -> 0
@@ -369,21 +417,32 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         // O is rescaled by the whole warp when any of its rows moved its max (alpha = 1
         // leaves the other rows unchanged); the first tile overwrites O instead.
         const bool rescale = n > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f);
-        float rowsum = 0.f;
+        const float2 neg_m2 = make_float2(-m_run, -m_run);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e]), p.scale_log2, -m_run));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e + 1]), p.scale_log2, -m_run));
-            rowsum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[c][2 * e]), __uint_as_float(r[c][2 * e + 1])),
+                                        scale2, neg_m2);
+            float2 pr;
+            if (c >= 4 - kPolyCols / 32) {
+              pr = exp2_poly2(x);
+            } else {
+              pr.x = ex2_approx(x.x);
+              pr.y = ex2_approx(x.y);
+            }
+            acc[e & 3] = __fadd2_rn(acc[e & 3], pr);
+            pk[e] = pack_bf16x2(pr.x, pr.y);
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[c][e] = pk[e];
         }
-        l_run += rowsum;
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+        const float2 a = __fadd2_rn(a01, a23);
+        l_run += a.x + a.y;
         if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {

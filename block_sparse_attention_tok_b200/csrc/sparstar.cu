@@ -23,6 +23,12 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxCandidates = 16384;  // Top-K keys held in shared memory (64 KB)
+// Columns of each 128-column S row whose exp2 runs on the FMA pipe instead of MUFU.
+#ifndef SPARSTAR_POLY_COLS
+#define SPARSTAR_POLY_COLS 0
+#endif
+constexpr int kPolyCols128 = SPARSTAR_POLY_COLS;
+constexpr int kPolyCols64 = SPARSTAR_POLY_COLS;
 
 struct DeviceInfo {
   bool ready = false;
@@ -71,9 +77,9 @@ int set_kernel_attrs(DeviceInfo* d) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (d->attrs_set) return SPARSTAR_OK;
   bool ok = true;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128, kPolyCols128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<128>::kSmemBytes) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, kPolyCols64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * 64 * (128 + 4) * 4) == cudaSuccess;
@@ -286,9 +292,9 @@ int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_
   const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (head_dim == 128)
-    attn_sparse_kernel<128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
+    attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
   else
-    attn_sparse_kernel<64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+    attn_sparse_kernel<64, kPolyCols64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
   return launch_status();
 }
 
