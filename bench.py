@@ -50,6 +50,37 @@ def parse():
     return ap.parse_args()
 
 
+KERNEL_SOURCES = ("attn_sm100.cuh", "ptx.cuh", "select.cuh", "sparstar.cu")
+
+
+def kernel_source_hash() -> str:
+    """sha256 (first 16 hex digits) of the CUDA sources the kernels are built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_attention_tok_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture of this exact source, else None.
+
+    profiles/traffic.txt lines: <source hash> <kernel> <workload> <bytes per launch> <note...>
+    """
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == want and parts[1] == kernel \
+                    and parts[2] == workload:
+                return float(parts[3])
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -126,6 +157,28 @@ def kept_tile_flops(idx: torch.Tensor, cnt: torch.Tensor, n_q: int, n_kv: int, d
     vq = torch.full((nqb,), 128.0, dtype=torch.float64, device=idx.device)
     vq[-1] = n_q - (nqb - 1) * 128
     return float(4.0 * d * (per_row * vq[None, :]).sum().item())
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def rank_seeds(sc, rank: int):
+    """Seeds of one rank's heads: every rank works on its own full scale (weak scaling)."""
+    return [1000 * synth.CFG_INDEX.get(sc.name, 0) + h + 100000 * rank for h in range(sc.heads)]
+
+
+def max_over_ranks(values, device, world: int):
+    """Elementwise max of per-rank timings (a no-op on one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Aggregate throughput: the units all ranks processed over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -221,8 +274,7 @@ def run_ours(args, rank, world, local_rank):
     sc = synth.WORKLOADS[args.workload]
     if args.heads:
         sc = dataclasses.replace(sc, heads=args.heads)
-    seeds = [1000 * synth.CFG_INDEX.get(sc.name, 0) + h + 100000 * rank for h in range(sc.heads)]
-    q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim, seeds, device=dev)
+    q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim, rank_seeds(sc, rank), device=dev)
     plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode)
     kmax = int(plan.k_total)
     ws = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
@@ -272,10 +324,7 @@ def run_ours(args, rank, world, local_rank):
     t_sel = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     status = S.device_status()
-    if world > 1:
-        t = torch.tensor([ms, t_sel, t_att], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, t_sel, t_att = (float(x) for x in t.tolist())
+    ms, t_sel, t_att = max_over_ranks([ms, t_sel, t_att], dev, world)
 
     peaks, peak_src = load_peaks()
     attn_tflops = flops / (t_att * 1e-3) / 1e12
@@ -284,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
     peak_hbm = float(peaks["hbm_gbs"])
     result = {
         "metric": METRIC,
-        "value": world * flops / (ms * 1e-3) / 1e12,
+        "value": whole_job_tflops(flops, ms, world),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -296,7 +345,8 @@ def run_ours(args, rank, world, local_rank):
                    "bytes": sel_bytes, "share_of_step": t_sel / (t_sel + t_att)},
         "us_per_scale": ms * 1e3,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak_t, "traffic": None,
+                     "frac": attn_tflops / peak_t,
+                     "traffic": recorded_traffic("attn_sparse_kernel<128>", sc.name if not args.heads else ""),
                      "kernel": "attn_sparse_kernel<128>",
                      "peak_source": f"{peak_src} bf16 sustained (kernel inside a back-to-back step loop)"},
         "device_status": int(status),
@@ -345,12 +395,8 @@ def run_ours(args, rank, world, local_rank):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        result["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+        ems, = max_over_ranks([a.elapsed_time(b) / n_e2e], dev, world)
+        result["e2e"] = {"value": whole_job_tflops(flops, ems, world), "unit": "TFLOP/s",
                          "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                          "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e}
         del hq, hk, hv, ho
