@@ -5,20 +5,27 @@
 // key block) pair gets an aggregate score from the pooled vectors, the clip-aware forced
 // blocks are kept, and the rest of each row is filled by a joint Top-K, per head.
 //
-// Kernels (all fp32 arithmetic on bf16 inputs):
-//   pool_kernel   one CTA per 128-token block: 16-byte streaming loads, fp32 sums,
-//                 shuffle + shared-memory reduction, divide by the valid token count.
-//   score_kernel  64x64 tiles of S = qbar kbar^T * (1/sqrt(d)) per head, fp32 FFMA with a
-//                 4x4 register tile per thread.
-//   topk_kernel   one CTA per (head, query block) row: order-preserving 32-bit keys,
-//                 8-bit MSB radix select of the K-th largest key, ties at the threshold
-//                 taken lowest index first, ascending emit after the forced prefix.
-//   fill_kernel   rows that do not depend on scores (K_topk == 0 or every block kept):
-//                 the row is the identity prefix 0..K_total-1.
+// Kernels:
+//   pool_kernel      one CTA per 128-token block: 16-byte streaming loads, fp32 sums,
+//                    shuffle + shared-memory reduction, divide by the valid token count; the
+//                    mean m is stored as two bf16 numbers hi = bf16(m), lo = bf16(m - hi).
+//   score_tc_kernel  S = qbar kbar^T / sqrt(d) on the tensor cores: per CTA a 128 x 256 tile
+//                    of (query block, KV block) pairs, TMA-fed, tcgen05.mma accumulating
+//                    hi.hi + hi.lo + lo.hi in fp32 tensor memory (the dropped lo.lo term and
+//                    the bf16 rounding of lo keep the error near 2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
+//   topk_warp_kernel one warp per (head, query block) row, keys in registers: the K-th largest
+//                    key is bracketed by counting, then resolved among <= 32 keys by a warp
+//                    bitonic sort; ties taken lowest index first, ascending emit.
+//   topk_kernel      one CTA per row, 8-bit radix select in shared memory (rows with more than
+//                    2048 candidates).
+//   fill_kernel      rows that do not depend on scores (K_topk == 0 or every block kept):
+//                    the row is the identity prefix 0..K_total-1.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
+
+#include "ptx.cuh"
 
 namespace sparstar {
 
@@ -42,12 +49,13 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
 }
 
 // grid.x = H * (nq_blocks + nk_blocks) (Q blocks of a head first, then its K blocks);
-// nq_blocks may be 0 (pool K only). 256 threads.
+// nq_blocks may be 0 (pool K only). 256 threads. Outputs [H, n_blocks, D] bf16 hi and lo.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, int64_t n_q,
                                                    int64_t n_kv, int nq_blocks, int nk_blocks,
-                                                   float* __restrict__ qbar, float* __restrict__ kbar) {
+                                                   __nv_bfloat16* __restrict__ q_hi, __nv_bfloat16* __restrict__ q_lo,
+                                                   __nv_bfloat16* __restrict__ k_hi, __nv_bfloat16* __restrict__ k_lo) {
   constexpr int kChunks = D / 8;           // 16-byte chunks per token row
   constexpr int kRowGroups = 256 / kChunks;
   constexpr int kRowsPerThread = 128 / kRowGroups;
@@ -57,19 +65,23 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int h = blockIdx.x / per_head;
   const int r = blockIdx.x - h * per_head;
   const __nv_bfloat16* src;
-  float* dst;
+  __nv_bfloat16 *dst_hi, *dst_lo;
   int64_t n_tok;
   int64_t b;
   if (r < nq_blocks) {
     b = r;
     n_tok = n_q;
     src = q + static_cast<int64_t>(h) * n_q * D;
-    dst = qbar + (static_cast<int64_t>(h) * nq_blocks + b) * D;
+    const int64_t o = (static_cast<int64_t>(h) * nq_blocks + b) * D;
+    dst_hi = q_hi + o;
+    dst_lo = q_lo + o;
   } else {
     b = r - nq_blocks;
     n_tok = n_kv;
     src = k + static_cast<int64_t>(h) * n_kv * D;
-    dst = kbar + (static_cast<int64_t>(h) * nk_blocks + b) * D;
+    const int64_t o = (static_cast<int64_t>(h) * nk_blocks + b) * D;
+    dst_hi = k_hi + o;
+    dst_lo = k_lo + o;
   }
   const int64_t row0 = b * 128;
   const int n_valid = static_cast<int>(min(static_cast<int64_t>(128), n_tok - row0));
@@ -101,67 +113,138 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
-    dst[threadIdx.x] = s / static_cast<float>(n_valid);
+    const float m = s / static_cast<float>(n_valid);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(m);
+    dst_hi[threadIdx.x] = hi;
+    dst_lo[threadIdx.x] = __float2bfloat16_rn(m - __bfloat162float(hi));
   }
 }
 
 // ------------------------------------------------------------------------ scores
 
-// grid = (ceil(nkb/64), ceil(nqb/64), H); 256 threads; dynamic smem 2*64*(D+4) floats.
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                                    int nqb, int nkb, float inv_sqrt_d, float* __restrict__ S) {
-  constexpr int LD = D + 4;
-  extern __shared__ __align__(16) float smem_f[];
-  float* qs = smem_f;
-  float* ks = smem_f + 64 * LD;
-  const int h = blockIdx.z;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
-  const float* qh = qbar + static_cast<int64_t>(h) * nqb * D;
-  const float* kh = kbar + static_cast<int64_t>(h) * nkb * D;
-  constexpr int kVec = 64 * D / 4;
-  for (int e = threadIdx.x; e < kVec; e += 256) {
-    const int row = e / (D / 4), c4 = e % (D / 4);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (i0 + row < nqb) a = *reinterpret_cast<const float4*>(qh + static_cast<int64_t>(i0 + row) * D + c4 * 4);
-    if (j0 + row < nkb) b = *reinterpret_cast<const float4*>(kh + static_cast<int64_t>(j0 + row) * D + c4 * 4);
-    *reinterpret_cast<float4*>(qs + row * LD + c4 * 4) = a;
-    *reinterpret_cast<float4*>(ks + row * LD + c4 * 4) = b;
+struct ScoreConfig {
+  static constexpr int kChunks = D / 64;                    // 128-byte swizzle chunks per row
+  static constexpr uint32_t kQChunk = 128 * 128;            // 128 query-block rows x 128 B
+  static constexpr uint32_t kKChunk = 256 * 128;            // 256 KV-block rows x 128 B
+  static constexpr uint32_t kQBytes = kChunks * kQChunk;    // hi (or lo) tile of qbar
+  static constexpr uint32_t kKBytes = kChunks * kKChunk;    // hi (or lo) tile of kbar
+  static constexpr uint32_t kOperandBytes = 2 * kQBytes + 2 * kKBytes;
+  static constexpr uint32_t kStageRow = 260;                // floats per staged S row (256 + pad)
+  static constexpr uint32_t kStageBytes = 128 * kStageRow * 4;
+  // Operands and the epilogue's staging area share one region (used one after the other).
+  static constexpr uint32_t kDataBytes = kOperandBytes > kStageBytes ? kOperandBytes : kStageBytes;
+  static constexpr uint32_t kSmemBytes = 1024 + kDataBytes + 64;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);
+  static constexpr uint32_t kTmemCols = 256;
+};
+
+// grid = (ceil(nkb/256), ceil(nqb/128), H); 128 threads. One elected thread loads the four
+// tiles with TMA (out-of-range rows are zero) and issues 3 * D/16 MMAs of M=128, N=256, K=16;
+// each warp then reads its 32 rows of the fp32 accumulator and writes S.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_ql,
+                    const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kl,
+                    float* __restrict__ S, int nqb, int nkb, float inv_sqrt_d, unsigned* status) {
+  using C = ScoreConfig<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* qh_s = smem;
+  uint8_t* ql_s = qh_s + C::kQBytes;
+  uint8_t* kh_s = ql_s + C::kQBytes;
+  uint8_t* kl_s = kh_s + C::kKBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kDataBytes);
+  uint64_t* done = full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.z, i0 = blockIdx.y * 128, j0 = blockIdx.x * 256;
+
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
   }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4];
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(full, 2 * C::kQBytes + 2 * C::kKBytes);
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+    for (int c = 0; c < C::kChunks; ++c) {
+      tma_load_3d(smem_u32(qh_s + c * C::kQChunk), &tm_qh, full, c * 64, i0, h);
+      tma_load_3d(smem_u32(ql_s + c * C::kQChunk), &tm_ql, full, c * 64, i0, h);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < D; c += 4) {
-    float4 av[4], bv[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) av[a] = *reinterpret_cast<const float4*>(qs + (ty + 16 * a) * LD + c);
-#pragma unroll
-    for (int b = 0; b < 4; ++b) bv[b] = *reinterpret_cast<const float4*>(ks + (tx + 16 * b) * LD + c);
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        acc[a][b] = fmaf(av[a].x, bv[b].x, acc[a][b]);
-        acc[a][b] = fmaf(av[a].y, bv[b].y, acc[a][b]);
-        acc[a][b] = fmaf(av[a].z, bv[b].z, acc[a][b]);
-        acc[a][b] = fmaf(av[a].w, bv[b].w, acc[a][b]);
+      for (int half = 0; half < 2; ++half) {
+        tma_load_3d(smem_u32(kh_s + c * C::kKChunk + half * 16384), &tm_kh, full, c * 64, j0 + 128 * half, h);
+        tma_load_3d(smem_u32(kl_s + c * C::kKChunk + half * 16384), &tm_kl, full, c * 64, j0 + 128 * half, h);
       }
-  }
-  float* Sh = S + static_cast<int64_t>(h) * nqb * nkb;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty + 16 * a;
-    if (i >= nqb) continue;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + tx + 16 * b;
-      if (j < nkb) Sh[static_cast<int64_t>(i) * nkb + j] = acc[a][b] * inv_sqrt_d;
     }
+    if (mbar_wait(full, 0, abort_flag, status)) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t qa = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
+        const uint32_t kb = (kk >> 2) * C::kKChunk + (kk & 3) * 32;
+        const uint64_t dqh = smem_desc_sw128(smem_u32(qh_s) + qa, 16, 1024);
+        const uint64_t dql = smem_desc_sw128(smem_u32(ql_s) + qa, 16, 1024);
+        const uint64_t dkh = smem_desc_sw128(smem_u32(kh_s) + kb, 16, 1024);
+        const uint64_t dkl = smem_desc_sw128(smem_u32(kl_s) + kb, 16, 1024);
+        mma_ss(tmem, dqh, dkh, C::kIdesc, kk > 0 ? 1u : 0u);
+        mma_ss(tmem, dqh, dkl, C::kIdesc, 1u);
+        mma_ss(tmem, dql, dkh, C::kIdesc, 1u);
+      }
+    }
+    mma_commit(done);  // also arrives when nothing was issued
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag, status));
+  tc_fence_after();
+  if (ok) {
+    // Stage this warp's 32 rows x 256 columns in the (now idle) operand buffers, padded to
+    // 260 floats per row so that the 16-byte stores of 32 rows hit distinct banks, then
+    // write whole row segments with coalesced stores.
+    float* stage = reinterpret_cast<float*>(smem) + warp * 32 * C::kStageRow;
+    float* my_row = stage + lane * C::kStageRow;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32 * c, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(my_row + 32 * c + e) =
+            make_float4(__uint_as_float(r[e]) * inv_sqrt_d, __uint_as_float(r[e + 1]) * inv_sqrt_d,
+                        __uint_as_float(r[e + 2]) * inv_sqrt_d, __uint_as_float(r[e + 3]) * inv_sqrt_d);
+    }
+    __syncwarp();
+    const int n_cols = min(256, nkb - j0);
+#pragma unroll 1
+    for (int rr = 0; rr < 32; ++rr) {
+      const int i = i0 + warp * 32 + rr;
+      if (i >= nqb) break;
+      float* srow = S + (static_cast<int64_t>(h) * nqb + i) * nkb + j0;
+      const float* src = stage + rr * C::kStageRow;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const int col = lane + 32 * cc;
+        if (col < n_cols) srow[col] = src[col];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -169,10 +252,9 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qb
 
 // Order-preserving key: larger score -> larger key; -0.0 maps like +0.0; NaN ranks last.
 __device__ __forceinline__ uint32_t score_key(float s) {
-  if (s != s) return 0u;
-  if (s == 0.0f) s = 0.0f;
-  const uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint32_t u = s == 0.0f ? 0u : __float_as_uint(s);  // -0.0 -> +0.0
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return s != s ? 0u : k;
 }
 
 // Exclusive prefix sum over the 128 threads of the block (4 warps); returns the total too.
@@ -301,6 +383,208 @@ __global__ void __launch_bounds__(128) fill_kernel(int k_total, int32_t* __restr
   const int64_t row = blockIdx.x;
   for (int c = threadIdx.x; c < k_total; c += 128) idx[row * kmax + c] = c;
   if (threadIdx.x == 0) cnt[row] = k_total;
+}
+
+// Top-K of one row by one warp; the row's scores sit in this warp's shared-memory buffer
+// sv[32 * KPL]. The K-th largest key T is located in steps, all exact:
+//   1. the row's score range is split into 256 equal-width bins; binning is monotone in the
+//      score, so every key in a higher bin is larger than every key in a lower one;
+//   2. a per-warp histogram (`hist`, 256 words) and a warp scan give the bin b* holding the
+//      K-th largest key and the number of keys above it;
+//   3. the indices of the keys in bins >= b* (about K of them) are compacted in index order
+//      into `lst` (uint16, one per candidate at most); every later step reads only this list;
+//   4. the keys of b* are gathered (`gather`, 32 words) and sorted by a warp bitonic network;
+//      if b* holds more than 32 keys, its key range is first narrowed by bisection on counts.
+// Every key > T is taken, and of the keys == T the lowest-index ones; the row is emitted
+// ascending after the forced prefix. Keys: NaN ranks below every number; -0.0 equals +0.0.
+template <int KPL>
+__device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, int n_forced, int n_cand, int k_topk,
+                                              int32_t* __restrict__ out, uint32_t* gather, uint32_t* hist,
+                                              float* sv, uint16_t* lst) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t full = 0xFFFFFFFFu;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const uint32_t K = static_cast<uint32_t>(k_topk);
+  // Row -> shared memory with asynchronous 4-byte copies (nothing held in registers).
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    const int j = lane + 32 * t;
+    if (j < n_cand)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sv + j)), "l"(srow + n_forced + j)
+                   : "memory");
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncwarp();
+  auto key_of = [](float x) -> uint32_t { return x != x ? 1u : max(score_key(x), 2u); };
+  // 1. score range (fminf/fmaxf skip NaN)
+  float lo_s[4] = {INFINITY, INFINITY, INFINITY, INFINITY}, hi_s[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    if (lane + 32 * t < n_cand) {
+      const float x = sv[lane + 32 * t];
+      lo_s[t & 3] = fminf(lo_s[t & 3], x);
+      hi_s[t & 3] = fmaxf(hi_s[t & 3], x);
+    }
+  }
+  float smin = fminf(fminf(lo_s[0], lo_s[1]), fminf(lo_s[2], lo_s[3]));
+  float smax = fmaxf(fmaxf(hi_s[0], hi_s[1]), fmaxf(hi_s[2], hi_s[3]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    smin = fminf(smin, __shfl_xor_sync(full, smin, off));
+    smax = fmaxf(smax, __shfl_xor_sync(full, smax, off));
+  }
+  const float width = smax - smin;
+  const float scale = width > 0.f ? 256.f / width : 0.f;
+  const float offset = -smin * scale;
+  auto bin_of = [&](float x) -> uint32_t {  // monotone in x; NaN -> 0
+    const float f = fmaf(x, scale, offset);
+    return f != f ? 0u : min(255u, __float2uint_rz(f));
+  };
+  // 2. histogram and the bin of the K-th largest key
+#pragma unroll
+  for (int t = 0; t < KPL; ++t)
+    if (lane + 32 * t < n_cand) atomicAdd(&hist[bin_of(sv[lane + 32 * t])], 1u);
+  __syncwarp();
+  uint32_t cnt[8], local = 0;  // lane l owns bins 255-8l .. 248-8l (descending)
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    cnt[e] = hist[255 - 8 * lane - e];
+    local += cnt[e];
+  }
+  uint32_t inc = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t n = __shfl_up_sync(full, inc, off);
+    if (lane >= off) inc += n;
+  }
+  uint32_t before = inc - local;
+  const bool owner = before < K && K <= inc;
+  uint32_t bstar_l = 0, above_l = 0, inbin_l = 0;
+  if (owner) {
+    bool done = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (!done && before + cnt[e] >= K) {
+        bstar_l = 255u - 8u * lane - e;
+        above_l = before;
+        inbin_l = cnt[e];
+        done = true;
+      }
+      before += cnt[e];
+    }
+  }
+  const int src = __ffs(__ballot_sync(full, owner)) - 1;
+  const uint32_t bstar = __shfl_sync(full, bstar_l, src);
+  uint32_t c_hi = __shfl_sync(full, above_l, src);          // #(keys in bins above b*)
+  uint32_t c_lo = c_hi + __shfl_sync(full, inbin_l, src);   // #(keys in bins >= b*)
+  // 3. compact the indices with bin >= b*, in index order
+  uint32_t m = 0;
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    const int j = lane + 32 * t;
+    const bool in = j < n_cand && bin_of(sv[j]) >= bstar;
+    const uint32_t ball = __ballot_sync(full, in);
+    if (in) lst[m + __popc(ball & lt_mask)] = static_cast<uint16_t>(j);
+    m += __popc(ball);
+  }
+  __syncwarp();
+  // 4. key range of b*, narrowed while it holds more than 32 keys
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (uint32_t e = lane; e < m; e += 32) {
+    const float x = sv[lst[e]];
+    if (bin_of(x) == bstar) {
+      const uint32_t k = key_of(x);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+  }
+  uint64_t lo = __reduce_min_sync(full, kmin);
+  uint64_t hi = static_cast<uint64_t>(__reduce_max_sync(full, kmax)) + 1u;
+  while (c_lo - c_hi > 32u && hi - lo > 1u) {
+    const uint64_t mid = lo + ((hi - lo) >> 1);
+    uint32_t c = 0;
+    for (uint32_t e = lane; e < m; e += 32) c += key_of(sv[lst[e]]) >= static_cast<uint32_t>(mid) ? 1u : 0u;
+    const uint32_t cm = __reduce_add_sync(full, c);
+    if (cm >= K) {
+      lo = mid;
+      c_lo = cm;
+    } else {
+      hi = mid;
+      c_hi = cm;
+    }
+  }
+  uint32_t base = 0;
+  for (uint32_t e0 = 0; e0 < m; e0 += 32) {
+    const uint32_t e = e0 + lane;
+    const uint32_t k = e < m ? key_of(sv[lst[e]]) : 0u;
+    const bool in = e < m && k >= lo && static_cast<uint64_t>(k) < hi;
+    const uint32_t ball = __ballot_sync(full, in);
+    const uint32_t at = base + __popc(ball & lt_mask);
+    if (in && at < 32u) gather[at] = k;
+    base += __popc(ball);
+  }
+  __syncwarp();
+  uint32_t g = lane < static_cast<int>(min(base, 32u)) ? gather[lane] : 0u;
+  __syncwarp();
+#pragma unroll
+  for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      const uint32_t other = __shfl_xor_sync(full, g, jj);
+      const bool descending_block = (lane & kk) == 0;
+      const bool first = (lane & jj) == 0;
+      g = (first == descending_block) ? max(g, other) : min(g, other);
+    }
+  }
+  // need-th largest inside the range (1 <= need <= 32 because c_lo >= K > c_hi); a range
+  // narrowed to one key value (possibly held by more than 32 candidates) is T itself.
+  const uint32_t need = K - c_hi;
+  const uint32_t T_sorted = __shfl_sync(full, g, static_cast<int>(min(need, 32u)) - 1);
+  const uint32_t T = (hi - lo == 1u) ? static_cast<uint32_t>(lo) : T_sorted;
+  // 5. emit: every listed key > T and the lowest-index keys == T, in index order
+  uint32_t n_gt = 0;
+  for (uint32_t e = lane; e < m; e += 32) n_gt += key_of(sv[lst[e]]) > T ? 1u : 0u;
+  const uint32_t need_eq = K - __reduce_add_sync(full, n_gt);
+  for (int f = lane; f < n_forced; f += 32) out[f] = f;
+  uint32_t pos = static_cast<uint32_t>(n_forced), eq_seen = 0;
+  const uint32_t row_end = static_cast<uint32_t>(n_forced + k_topk);
+  for (uint32_t e0 = 0; e0 < m; e0 += 32) {
+    const uint32_t e = e0 + lane;
+    const uint32_t j = e < m ? lst[e] : 0u;
+    const uint32_t k = e < m ? key_of(sv[j]) : 0u;
+    const uint32_t eq_ball = __ballot_sync(full, e < m && k == T);
+    const bool take = e < m && (k > T || (k == T && eq_seen + __popc(eq_ball & lt_mask) < need_eq));
+    eq_seen += __popc(eq_ball);
+    const uint32_t take_ball = __ballot_sync(full, take);
+    const uint32_t at = pos + __popc(take_ball & lt_mask);
+    if (take && at < row_end) out[at] = n_forced + static_cast<int>(j);
+    pos += __popc(take_ball);
+  }
+}
+
+template <int KPL>
+constexpr int topk_warp_smem() {
+  return 8 * 32 * KPL * (4 + 2);  // per warp: scores (fp32) and the compacted index list (uint16)
+}
+
+// One warp per row, 8 rows per 256-thread CTA; grid.x = ceil(H * nqb / 8). Requires
+// 1 <= k_topk < n_cand <= 32 * KPL.
+template <int KPL>
+__global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict__ S, int64_t rows, int nkb,
+                                                        int n_forced, int k_topk, int32_t* __restrict__ idx,
+                                                        int32_t* __restrict__ cnt, int kmax) {
+  __shared__ uint32_t gather[8][32];
+  __shared__ uint32_t hist[8][256];
+  extern __shared__ float rowbuf[];  // [8][32 * KPL] scores, then [8][32 * KPL] uint16 lists
+  const int w = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + w;
+  if (row >= rows) return;
+  uint16_t* lists = reinterpret_cast<uint16_t*>(rowbuf + 8 * 32 * KPL);
+  topk_row_warp<KPL>(S + row * nkb, n_forced, nkb - n_forced, k_topk, idx + row * kmax, gather[w], hist[w],
+                     rowbuf + w * 32 * KPL, lists + w * 32 * KPL);
+  if ((threadIdx.x & 31) == 0) cnt[row] = n_forced + k_topk;
 }
 
 }  // namespace sparstar

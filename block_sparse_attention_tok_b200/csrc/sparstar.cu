@@ -81,10 +81,16 @@ int set_kernel_attrs(DeviceInfo* d) {
                              AttnConfig<128>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, kPolyCols64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64>::kSmemBytes) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * 64 * (128 + 4) * 4) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ScoreConfig<128>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ScoreConfig<64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMaxCandidates * 4)) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(topk_warp_kernel<36>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             topk_warp_smem<36>()) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(topk_warp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             topk_warp_smem<64>()) == cudaSuccess;
   if (!ok) return SPARSTAR_ERR_CUDA;
   d->attrs_set = true;
   return SPARSTAR_OK;
@@ -101,17 +107,34 @@ bool valid_segments(const sparstar_segments& s) { return s.n_text >= 0 && s.n_ct
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
+int launch_status() { return cudaGetLastError() == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ERR_CUDA; }
+
+// Workspace: [q_hi | q_lo] [k_hi | k_lo] [scores]: the block means as bf16 hi/lo pairs
+// ([H, n_blocks, d] each) and the fp32 score matrix [H, nqb, nkb].
 struct Workspace {
-  size_t qbar, kbar, scores, total;
+  size_t q_hi, q_lo, k_hi, k_lo, scores, total;
 };
 
 Workspace workspace_layout(int heads, int64_t nqb, int64_t nkb, int d, bool need_scores) {
   Workspace w;
-  w.qbar = 0;
-  w.kbar = align256(static_cast<size_t>(heads) * nqb * d * sizeof(float));
-  w.scores = w.kbar + align256(static_cast<size_t>(heads) * nkb * d * sizeof(float));
+  const size_t qb = static_cast<size_t>(heads) * nqb * d * 2, kb = static_cast<size_t>(heads) * nkb * d * 2;
+  w.q_hi = 0;
+  w.q_lo = align256(qb);
+  w.k_hi = w.q_lo + align256(qb);
+  w.k_lo = w.k_hi + align256(kb);
+  w.scores = w.k_lo + align256(kb);
   w.total = w.scores + (need_scores ? align256(static_cast<size_t>(heads) * nqb * nkb * sizeof(float)) : 0);
   return w;
+}
+
+// Keys per lane of the warp Top-K: the smallest supported count that covers n_cand
+// candidates, or 0 when the shared-memory radix kernel has to be used.
+int topk_keys_per_lane(int64_t n_cand) {
+  if (n_cand <= 32 * 8) return 8;
+  if (n_cand <= 32 * 16) return 16;
+  if (n_cand <= 32 * 36) return 36;
+  if (n_cand <= 32 * 64) return 64;
+  return 0;
 }
 
 int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d) {
@@ -126,7 +149,6 @@ int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d)
   return r == CUDA_SUCCESS ? SPARSTAR_OK : SPARSTAR_ERR_CUDA;
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ERR_CUDA; }
 
 }  // namespace
 }  // namespace sparstar
@@ -222,28 +244,56 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
   const int nqb = static_cast<int>(plan.nqb), nkb = static_cast<int>(plan.nkb);
 
   if (compute_scores) {
+    if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;  // tensor-core scores need sm_100
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
-    float* qbar = reinterpret_cast<float*>(wsb + ws.qbar);
-    float* kbar = reinterpret_cast<float*>(wsb + ws.kbar);
+    auto* q_hi = reinterpret_cast<__nv_bfloat16*>(wsb + ws.q_hi);
+    auto* q_lo = reinterpret_cast<__nv_bfloat16*>(wsb + ws.q_lo);
+    auto* k_hi = reinterpret_cast<__nv_bfloat16*>(wsb + ws.k_hi);
+    auto* k_lo = reinterpret_cast<__nv_bfloat16*>(wsb + ws.k_lo);
     float* S = scores != nullptr ? scores : reinterpret_cast<float*>(wsb + ws.scores);
+    CUtensorMap tqh, tql, tkh, tkl;
+    if (make_map(&tqh, q_hi, nqb, heads, head_dim) != SPARSTAR_OK ||
+        make_map(&tql, q_lo, nqb, heads, head_dim) != SPARSTAR_OK ||
+        make_map(&tkh, k_hi, nkb, heads, head_dim) != SPARSTAR_OK ||
+        make_map(&tkl, k_lo, nkb, heads, head_dim) != SPARSTAR_OK)
+      return SPARSTAR_ERR_CUDA;
     const unsigned pool_grid = static_cast<unsigned>(heads) * static_cast<unsigned>(nqb + nkb);
-    const dim3 sgrid((nkb + 63) / 64, (nqb + 63) / 64, heads);
+    const dim3 sgrid((nkb + 255) / 256, (nqb + 127) / 128, heads);
     const float inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(head_dim));
     if (head_dim == 128) {
       pool_kernel<128><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, qbar,
-                                                  kbar);
-      score_kernel<128><<<sgrid, 256, 2 * 64 * (128 + 4) * 4, st>>>(qbar, kbar, nqb, nkb, inv_sqrt_d, S);
+                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
+                                                  q_lo, k_hi, k_lo);
+      score_tc_kernel<128><<<sgrid, 128, ScoreConfig<128>::kSmemBytes, st>>>(tqh, tql, tkh, tkl, S, nqb, nkb,
+                                                                             inv_sqrt_d, dev->status);
     } else {
       pool_kernel<64><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                 static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, qbar,
-                                                 kbar);
-      score_kernel<64><<<sgrid, 256, 2 * 64 * (64 + 4) * 4, st>>>(qbar, kbar, nqb, nkb, inv_sqrt_d, S);
+                                                 static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
+                                                 q_lo, k_hi, k_lo);
+      score_tc_kernel<64><<<sgrid, 128, ScoreConfig<64>::kSmemBytes, st>>>(tqh, tql, tkh, tkl, S, nqb, nkb,
+                                                                           inv_sqrt_d, dev->status);
     }
     if ((rc = launch_status()) != SPARSTAR_OK) return rc;
     if (needs_scores) {
-      topk_kernel<<<static_cast<unsigned>(rows), 128, static_cast<size_t>(plan.n_cand) * 4, st>>>(
-          S, nkb, static_cast<int>(plan.n_forced), plan.k_topk, idx, cnt, kmax);
+      const int n_forced = static_cast<int>(plan.n_forced);
+      const unsigned tgrid = static_cast<unsigned>((rows + 7) / 8);
+      switch (topk_keys_per_lane(plan.n_cand)) {
+        case 8:
+          topk_warp_kernel<8><<<tgrid, 256, topk_warp_smem<8>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          break;
+        case 16:
+          topk_warp_kernel<16><<<tgrid, 256, topk_warp_smem<16>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          break;
+        case 36:
+          topk_warp_kernel<36><<<tgrid, 256, topk_warp_smem<36>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          break;
+        case 64:
+          topk_warp_kernel<64><<<tgrid, 256, topk_warp_smem<64>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          break;
+        default:
+          topk_kernel<<<static_cast<unsigned>(rows), 128, static_cast<size_t>(plan.n_cand) * 4, st>>>(
+              S, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+      }
       return launch_status();
     }
   }

@@ -91,8 +91,9 @@ int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double dens
                        int budget_mode, sparstar_plan* out);
 
 /* Host only. Bytes of device workspace that sparstar_select / sparstar_forward need for
- * these sizes (pooled block means and, unless the caller passes `scores`, the score
- * matrix). Writes *bytes; returns SPARSTAR_ERR_ARG on bad sizes. */
+ * these sizes (the pooled block means, each stored as a bf16 hi/lo pair, and, unless the
+ * caller passes `scores`, the fp32 score matrix). Writes *bytes; returns SPARSTAR_ERR_ARG
+ * on bad sizes. */
 int sparstar_workspace_size(int heads, int64_t n_q, sparstar_segments seg, int head_dim,
                             size_t* bytes);
 

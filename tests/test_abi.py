@@ -59,11 +59,12 @@ def test_plan_matches_oracle_budget(lib, n_q, n_text, n_ctx, n_cur, clip, densit
 
 
 def test_workspace_size(lib):
-    # pooled q (H*nqb*d), pooled k (H*nkb*d) and scores (H*nqb*nkb), fp32, 256-byte aligned
+    # pooled q and k as bf16 hi/lo pairs (2 x H*n_blocks*d x 2 B each) and fp32 scores
+    # (H*nqb*nkb), each section 256-byte aligned
     got = sparstar.workspace_size(32, 72192, 512, 72192, 72192, 128)
     def al(x):
         return (x + 255) // 256 * 256
-    assert got == al(32 * 564 * 128 * 4) + al(32 * 1132 * 128 * 4) + al(32 * 564 * 1132 * 4)
+    assert got == 2 * al(32 * 564 * 128 * 2) + 2 * al(32 * 1132 * 128 * 2) + al(32 * 564 * 1132 * 4)
 
 
 @pytest.mark.parametrize("kwargs,code", [
