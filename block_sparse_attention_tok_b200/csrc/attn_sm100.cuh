@@ -297,77 +297,92 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      SlotSeq seq0, seq1;
-      seq_init(seq0, blockIdx.x * 2 + 0, p, false);
-      seq_init(seq1, blockIdx.x * 2 + 1, p, false);
-      uint32_t ring_it = 0;
-      uint32_t tiles0 = 0u, tiles1 = 0u;
-      bool ok = true;
+    // The whole warp runs the schedule (waits and bookkeeping are warp-uniform, so addresses
+    // and descriptors stay in uniform registers); one elected lane issues each batch of
+    // tcgen05.mma / tcgen05.commit. Issue cost, not tensor time, bounds a lane-0-only loop.
+    SlotSeq seq0, seq1;
+    seq_init(seq0, blockIdx.x * 2 + 0, p, false);
+    seq_init(seq1, blockIdx.x * 2 + 1, p, false);
+    uint32_t ring_it = 0;
+    uint32_t tiles0 = 0u, tiles1 = 0u;
+    bool ok = true;
+    // A descriptor's start field is addr >> 4 in 14 bits; shared-memory addresses stay below
+    // 2^18, so desc(addr + off) = desc(addr) + (off >> 4) for 16-byte multiples off.
+    const uint64_t q_desc = smem_desc_sw128(smem_u32(q_tile), 16, 1024);
+    const uint64_t k_desc = smem_desc_sw128(smem_u32(ring), 16, 1024);
+    const uint64_t v_desc = smem_desc_sw128(smem_u32(ring), C::kChunkBytes, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, p.status));
+    };
 
-      auto issue_s = [&](int s, const SlotSeq& sq) -> bool {
-        if (sq.n == 0 && !mbar_wait(&q_full[s], sq.k & 1, abort_flag, p.status)) return false;
-        const uint32_t stage = ring_it % C::kStages;
-        if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(q_tile + s * C::kTileBytes);
-        const uint32_t ka = smem_u32(ring + stage * C::kTileBytes);
-        const uint32_t d_tmem = tmem_base + C::kTmemS + 128u * s;
+    // Q and K/V stages are filled by TMA: their mbarrier completion orders the tensor core's
+    // reads, so no tcgen05 fence is needed after those waits.
+    auto issue_s = [&](int s, const SlotSeq& sq) -> bool {
+      if (sq.n == 0 && !wait_all(&q_full[s], sq.k & 1)) return false;
+      const uint32_t stage = ring_it % C::kStages;
+      if (!wait_all(&full[stage], (ring_it / C::kStages) & 1u)) return false;
+      const uint64_t qd = q_desc + ((s * C::kTileBytes) >> 4);
+      const uint64_t kd = k_desc + ((stage * C::kTileBytes) >> 4);
+      const uint32_t d_tmem = tmem_base + C::kTmemS + 128u * s;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), C::kIdescQK,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
         mma_commit(&s_full[s]);
         if (sq.n == sq.ntiles - 1) mma_commit(&q_empty[s]);
-        ++ring_it;
-        return true;
-      };
-      auto issue_pv = [&](int s, const SlotSeq& sq, uint32_t& tiles) -> bool {
-        if (!mbar_wait(&p_full[s], tiles & 1u, abort_flag, p.status)) return false;
-        ++tiles;
-        const uint32_t stage = ring_it % C::kStages;
-        if (!mbar_wait(&full[stage], (ring_it / C::kStages) & 1u, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t va = smem_u32(ring + stage * C::kTileBytes);
-        const uint32_t d_tmem = tmem_base + C::kTmemO + 128u * s;
-        const uint32_t a_tmem = tmem_base + C::kTmemS + 128u * s;
+      }
+      __syncwarp();
+      ++ring_it;
+      return true;
+    };
+    auto issue_pv = [&](int s, const SlotSeq& sq, uint32_t& tiles) -> bool {
+      if (!wait_all(&p_full[s], tiles & 1u)) return false;
+      ++tiles;
+      const uint32_t stage = ring_it % C::kStages;
+      if (!wait_all(&full[stage], (ring_it / C::kStages) & 1u)) return false;
+      tc_fence_after();  // P was written by the softmax warps with tcgen05.st
+      const uint64_t vd = v_desc + ((stage * C::kTileBytes) >> 4);
+      const uint32_t d_tmem = tmem_base + C::kTmemO + 128u * s;
+      const uint32_t a_tmem = tmem_base + C::kTmemS + 128u * s;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // P columns: 16 bf16 per K step = 8 packed 32-bit columns.
           // V tile is MN-major for this MMA: 64-element chunks of d at 16 KB (LBO), 8-row
           // groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
-          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
-                 (sq.n > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), C::kIdescPV, (sq.n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
         if (sq.n == sq.ntiles - 1) mma_commit(&o_full[s]);
-        ++ring_it;
-        return true;
-      };
-      // One step of a slot: O += P V for its current tile, then S of its next tile.
-      auto step = [&](int s, SlotSeq& sq, uint32_t& tiles) {
-        if (!ok || sq.item < 0) return;
-        ok = issue_pv(s, sq, tiles);
-        if (!ok) return;
-        seq_next(sq, stride, p, false);
-        if (sq.item < 0) return;
-        ok = issue_s(s, sq);
-      };
+      }
+      __syncwarp();
+      ++ring_it;
+      return true;
+    };
+    // One step of a slot: O += P V for its current tile, then S of its next tile.
+    auto step = [&](int s, SlotSeq& sq, uint32_t& tiles) {
+      if (!ok || sq.item < 0) return;
+      ok = issue_pv(s, sq, tiles);
+      if (!ok) return;
+      seq_next(sq, stride, p, false);
+      if (sq.item < 0) return;
+      ok = issue_s(s, sq);
+    };
 
-      if (seq0.item >= 0) ok = issue_s(0, seq0);
-      if (ok && seq1.item >= 0) ok = issue_s(1, seq1);
-      while (ok && (seq0.item >= 0 || seq1.item >= 0)) {
-        step(0, seq0, tiles0);
-        step(1, seq1, tiles1);
-      }
-      // Drain: all issued MMAs complete before TMEM is released.
-      mma_commit(drain);
-      const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-      }
+    if (seq0.item >= 0) ok = issue_s(0, seq0);
+    if (ok && seq1.item >= 0) ok = issue_s(1, seq1);
+    while (ok && (seq0.item >= 0 || seq1.item >= 0)) {
+      step(0, seq0, tiles0);
+      step(1, seq1, tiles1);
+    }
+    // Drain: all issued MMAs complete before TMEM is released.
+    if (elect_one()) mma_commit(drain);
+    __syncwarp();
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
     }
     __syncwarp();
   } else {

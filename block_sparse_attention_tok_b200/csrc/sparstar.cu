@@ -338,9 +338,9 @@ int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_
   p.n_items = static_cast<int>(heads * nqb);
   const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int slots_needed = (p.n_items + 1) / 2;
   const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (head_dim == 128)
     attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
   else
