@@ -112,6 +112,16 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization
+// may start while its predecessor in the stream is still running; griddep_wait() blocks
+// until that predecessor grid has completed and its writes are visible (a no-op for a
+// normally launched kernel). griddep_launch_dependents() lets the successor be scheduled
+// before this grid finishes; it does not make this grid's writes visible early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // One lane of a converged warp (the lowest active one) gets true. Work issued under it stays
 // warp-uniform to the compiler, unlike work under a lane-index test.
 __device__ __forceinline__ bool elect_one() {

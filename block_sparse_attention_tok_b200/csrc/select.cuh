@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   constexpr int kRowGroups = 256 / kChunks;
   constexpr int kRowsPerThread = 128 / kRowGroups;
   __shared__ float part[8][D];
+  griddep_launch_dependents();  // the score kernel may be scheduled early; it waits for this grid
 
   const int per_head = nq_blocks + nk_blocks;
   const int h = blockIdx.x / per_head;
@@ -175,6 +176,8 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+  griddep_wait();  // pooled means come from the preceding pool kernel
 
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(full, 2 * C::kQBytes + 2 * C::kKBytes);
@@ -292,6 +295,7 @@ __global__ void __launch_bounds__(128) topk_kernel(const float* __restrict__ S, 
   const int n_cand = nkb - n_forced;
   const int64_t row = blockIdx.x;
   const float* srow = S + row * nkb + n_forced;
+  griddep_wait();  // scores come from the preceding score kernel
   for (int j = threadIdx.x; j < n_cand; j += 128) keys[j] = score_key(srow[j]);
 
   uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k_topk);
@@ -580,6 +584,7 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict_
   extern __shared__ float rowbuf[];  // [8][32 * KPL] scores, then [8][32 * KPL] uint16 lists
   const int w = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + w;
+  griddep_wait();  // scores come from the preceding score kernel
   if (row >= rows) return;
   uint16_t* lists = reinterpret_cast<uint16_t*>(rowbuf + 8 * 32 * KPL);
   topk_row_warp<KPL>(S + row * nkb, n_forced, nkb - n_forced, k_topk, idx + row * kmax, gather[w], hist[w],

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "sparstar.h"
 #include "attn_sm100.cuh"
@@ -125,6 +126,25 @@ Workspace workspace_layout(int heads, int64_t nqb, int64_t nkb, int d, bool need
   w.scores = w.k_lo + align256(kb);
   w.total = w.scores + (need_scores ? align256(static_cast<size_t>(heads) * nqb * nkb * sizeof(float)) : 0);
   return w;
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled while the
+// previous kernel of the stream drains; it calls griddep_wait() before reading that
+// kernel's output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Keys per lane of the warp Top-K: the smallest supported count that covers n_cand
@@ -264,14 +284,14 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
       pool_kernel<128><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                   static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
                                                   q_lo, k_hi, k_lo);
-      score_tc_kernel<128><<<sgrid, 128, ScoreConfig<128>::kSmemBytes, st>>>(tqh, tql, tkh, tkl, S, nqb, nkb,
-                                                                             inv_sqrt_d, dev->status);
+      launch_after(score_tc_kernel<128>, sgrid, dim3(128), ScoreConfig<128>::kSmemBytes, st, tqh, tql, tkh, tkl, S, nqb,
+                   nkb, inv_sqrt_d, dev->status);
     } else {
       pool_kernel<64><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
                                                  q_lo, k_hi, k_lo);
-      score_tc_kernel<64><<<sgrid, 128, ScoreConfig<64>::kSmemBytes, st>>>(tqh, tql, tkh, tkl, S, nqb, nkb,
-                                                                           inv_sqrt_d, dev->status);
+      launch_after(score_tc_kernel<64>, sgrid, dim3(128), ScoreConfig<64>::kSmemBytes, st, tqh, tql, tkh, tkl, S, nqb,
+                   nkb, inv_sqrt_d, dev->status);
     }
     if ((rc = launch_status()) != SPARSTAR_OK) return rc;
     if (needs_scores) {
@@ -279,20 +299,24 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
       const unsigned tgrid = static_cast<unsigned>((rows + 7) / 8);
       switch (topk_keys_per_lane(plan.n_cand)) {
         case 8:
-          topk_warp_kernel<8><<<tgrid, 256, topk_warp_smem<8>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          launch_after(topk_warp_kernel<8>, dim3(tgrid), dim3(256), topk_warp_smem<8>(), st, S, rows, nkb, n_forced,
+                       plan.k_topk, idx, cnt, kmax);
           break;
         case 16:
-          topk_warp_kernel<16><<<tgrid, 256, topk_warp_smem<16>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          launch_after(topk_warp_kernel<16>, dim3(tgrid), dim3(256), topk_warp_smem<16>(), st, S, rows, nkb, n_forced,
+                       plan.k_topk, idx, cnt, kmax);
           break;
         case 36:
-          topk_warp_kernel<36><<<tgrid, 256, topk_warp_smem<36>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          launch_after(topk_warp_kernel<36>, dim3(tgrid), dim3(256), topk_warp_smem<36>(), st, S, rows, nkb, n_forced,
+                       plan.k_topk, idx, cnt, kmax);
           break;
         case 64:
-          topk_warp_kernel<64><<<tgrid, 256, topk_warp_smem<64>(), st>>>(S, rows, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          launch_after(topk_warp_kernel<64>, dim3(tgrid), dim3(256), topk_warp_smem<64>(), st, S, rows, nkb, n_forced,
+                       plan.k_topk, idx, cnt, kmax);
           break;
         default:
-          topk_kernel<<<static_cast<unsigned>(rows), 128, static_cast<size_t>(plan.n_cand) * 4, st>>>(
-              S, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
+          launch_after(topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(128), static_cast<size_t>(plan.n_cand) * 4, st,
+                       S, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
       }
       return launch_status();
     }

@@ -126,6 +126,16 @@ def test_many_items_per_slot(S):
     assert stats["rows"] == 8 * 91
 
 
+@pytest.mark.parametrize("d,heads", [(64, 10), (128, 9)])
+def test_many_heads_ragged_tail(S, d, heads):
+    """An odd number of heads (more than a few) with a ragged last query and KV block, every
+    row and every output compared."""
+    n_cur = 128 * 6 + 5
+    q, k, v = synth.make_qkv(n_cur, 256 + 512 + n_cur, heads, d, [300 + h for h in range(heads)], device="cuda")
+    stats = _run_case(S, q, k, v, 256, 512, n_cur, 2, 0.3, 0)
+    assert stats["rows"] == heads * 7
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_row_max_jump_in_some_rows_only(S, d):
     """Rows 0-15 of every query block meet a much larger logit in a late KV block, so their
