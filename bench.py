@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-schedule", action="store_true",
+                    help="skip the per-scale timing of the refined-scale schedule (4 scales x 36 layers)")
     return ap.parse_args()
 
 
@@ -264,6 +266,69 @@ def workload_config(sc, args):
             "l2": "no flush: inputs 3.5 GB per GPU > 126 MB L2", "parallelism": f"replicas x{args.gpus}"}
 
 
+def run_schedule(S, dev, stream, layers: int = 36):
+    """Per-scale time of the refined-scale schedule of one clip (Clip 1): for each of the four
+    sparsified scales and each layer, fresh seeded inputs (untimed), then selection +
+    attention timed with CUDA events on resident inputs. Both budget readings; plus one
+    density-1 (dense) attention per scale through the same kernel, for context."""
+    out = {"workload": "refined-scale schedule, Clip 1: 4 scales x %d layers x 32 heads, d 128" % layers,
+           "modes": {}, "dense_ms_per_layer": {}}
+    for mode in (0, 1):
+        rows = []
+        for si, sc in enumerate(synth.SCHEDULE_CLIP1):
+            plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode)
+            kmax = int(plan.k_total)
+            ws = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
+            idx = torch.empty(sc.heads, int(plan.nqb), kmax, dtype=torch.int32, device=dev)
+            cnt = torch.empty(sc.heads, int(plan.nqb), dtype=torch.int32, device=dev)
+            t_sel, t_att, flops = [], [], 0.0
+            for layer in range(layers):
+                q, k, v = synth.make_scale_inputs(sc, device=dev, layer=layer, scale_index=si)
+                o, lse = torch.empty_like(q), torch.empty(sc.heads, sc.n_q, dtype=torch.float32, device=dev)
+                seg = (sc.n_text, sc.n_ctx, sc.n_cur)
+                if layer == 0:  # warm-up of this shape
+                    S.select(q, k, *seg, sc.clip, sc.density, mode, workspace=ws, idx=idx, cnt=cnt)
+                    S.attn(q, k, v, idx, cnt, o=o, lse=lse)
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                torch.cuda.synchronize()
+                ev[0].record(stream)
+                S.select(q, k, *seg, sc.clip, sc.density, mode, workspace=ws, idx=idx, cnt=cnt)
+                ev[1].record(stream)
+                S.attn(q, k, v, idx, cnt, o=o, lse=lse)
+                ev[2].record(stream)
+                torch.cuda.synchronize()
+                t_sel.append(ev[0].elapsed_time(ev[1]))
+                t_att.append(ev[1].elapsed_time(ev[2]))
+                flops += kept_tile_flops(idx, cnt, sc.n_q, sc.n_kv, sc.head_dim)
+                if mode == 0 and layer == 0:
+                    dplan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, 1.0)
+                    didx = torch.arange(int(dplan.nkb), dtype=torch.int32, device=dev).expand(
+                        sc.heads, int(dplan.nqb), int(dplan.nkb)).contiguous()
+                    dcnt = torch.full((sc.heads, int(dplan.nqb)), int(dplan.nkb), dtype=torch.int32, device=dev)
+                    S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+                    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    d0.record(stream)
+                    S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+                    d1.record(stream)
+                    torch.cuda.synchronize()
+                    out["dense_ms_per_layer"][sc.name] = d0.elapsed_time(d1)
+                    del didx, dcnt
+                del q, k, v, o, lse
+            ms_total = float(np.sum(t_sel) + np.sum(t_att))
+            rows.append({"scale": sc.name, "n_q": sc.n_q, "n_kv": sc.n_kv, "density": sc.density,
+                         "k_total": int(plan.k_total), "k_topk": int(plan.k_topk),
+                         "ms_all_layers": ms_total, "us_per_layer": ms_total * 1e3 / layers,
+                         "select_us_per_layer": float(np.mean(t_sel)) * 1e3,
+                         "attn_us_per_layer": float(np.mean(t_att)) * 1e3,
+                         "attn_tflops": flops / (float(np.sum(t_att)) * 1e-3) / 1e12,
+                         "selection_share": float(np.sum(t_sel)) / ms_total})
+            del ws, idx, cnt
+        out["modes"]["literal" if mode == 0 else "candidates"] = {
+            "scales": rows, "ms_schedule": float(sum(r["ms_all_layers"] for r in rows))}
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     from block_sparse_attention_tok_b200 import sparstar as S
     import torch.distributed as dist
@@ -400,6 +465,11 @@ def run_ours(args, rank, world, local_rank):
                          "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                          "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e}
         del hq, hk, hv, ho
+
+    if world == 1 and not args.no_schedule and not args.heads:
+        del o, lse
+        torch.cuda.empty_cache()
+        result["schedule"] = run_schedule(S, dev, stream)
 
     if rank == 0 and not args.no_cpu_baseline:
         qc, kc, vc = (x[:2].cpu() for x in (q, k, v))
