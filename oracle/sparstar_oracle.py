@@ -263,10 +263,60 @@ def block_energy(q: np.ndarray, k: np.ndarray, qblock: int, key_blocks: Sequence
     return float(p[:, cols].sum() / (e - s))
 
 
+def kept_token_count(kept_blocks: Sequence[int], n_kv: int, block: int = BLOCK) -> int:
+    """Valid KV tokens in the listed blocks (a ragged last block counts its valid tokens)."""
+    return int(len(kept_token_index(kept_blocks, n_kv, block)))
+
+
+def dense_probabilities(q_rows: np.ndarray, k: np.ndarray, sm_scale: float | None = None) -> np.ndarray:
+    """Dense softmax rows P_tu = exp(l_tu) / sum_u exp(l_tu), l_tu = sm_scale * q_t . k_u."""
+    scale = 1.0 / math.sqrt(q_rows.shape[1]) if sm_scale is None else sm_scale
+    logits = (q_rows @ k.T) * scale
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def token_topk_bound(q_rows: np.ndarray, k: np.ndarray, budget, sm_scale: float | None = None) -> np.ndarray:
+    """Token-wise upper bound on the retained mass (digest section 关键结果与论文证据, bullet
+    跨尺度复用损失, Figure 3): for each query row, the largest dense softmax mass that any
+    `budget` key tokens can hold, i.e. the sum of the row's `budget` largest probabilities.
+    `budget` is one count for all rows or one per row; a block mask keeping `budget` tokens
+    can retain at most this much."""
+    p = dense_probabilities(q_rows, k, sm_scale)
+    srt = -np.sort(-p, axis=1)
+    b = np.broadcast_to(np.asarray(budget, dtype=np.int64), (p.shape[0],))
+    out = np.empty(p.shape[0])
+    for t in range(p.shape[0]):
+        out[t] = srt[t, :int(b[t])].sum()
+    return out
+
+
+def mass_report(q: np.ndarray, k: np.ndarray, rows: np.ndarray, qblocks: Sequence[int],
+                sm_scale: float | None = None, block: int = BLOCK):
+    """For each listed query block i with kept blocks rows[i]: the mean over its valid rows t of
+    the retained mass R_t (dense softmax mass on the kept tokens; eq. (5) of the CalibAtt notes
+    divided by nothing else) and of the token-wise bound U_t with the same token budget.
+    Returns (E [len(qblocks)], U [len(qblocks)], R rows, U rows) with the per-row arrays
+    concatenated in qblocks order."""
+    E, U, R_rows, U_rows = [], [], [], []
+    for i in qblocks:
+        s, e = block_token_range(int(i), q.shape[0], block)
+        tokens = kept_token_index(rows[i], k.shape[0], block)
+        p = dense_probabilities(q[s:e], k, sm_scale)
+        r = p[:, tokens].sum(axis=1)
+        u = token_topk_bound(q[s:e], k, len(tokens), sm_scale)
+        E.append(r.mean())
+        U.append(u.mean())
+        R_rows.append(r)
+        U_rows.append(u)
+    return np.array(E), np.array(U), np.concatenate(R_rows), np.concatenate(U_rows)
+
+
 __all__ = [
     "BLOCK", "BUDGET_LITERAL", "BUDGET_CANDIDATES", "bf16_bits_to_f64", "num_blocks",
     "block_token_range", "forced_block_count", "row_budget", "pool_blocks", "block_scores",
     "select_rows", "select_row", "select_head", "select", "kept_token_index", "attend_rows",
     "block_sparse_attention", "dense_attention", "retained_mass", "block_energy",
+    "kept_token_count", "dense_probabilities", "token_topk_bound", "mass_report",
 ]
 

@@ -306,3 +306,58 @@ def test_heads_are_independent():
     perm = [2, 0, 1]
     idx_p, S_p = O.select(_bits(q[perm]), _bits(k[perm]), 128, 128, 2, 0.5)
     assert np.array_equal(idx_p, idx[perm]) and np.array_equal(S_p, S[perm])
+
+
+# ---------------------------------------------------------------- token-wise bound and mass
+
+def test_token_bound_equals_best_subset_bruteforce():
+    """The bound is the best mass over every key subset of the budget's size (enumerated)."""
+    rng = np.random.default_rng(71)
+    q = rng.normal(size=(3, 8))
+    k = rng.normal(size=(10, 8)) * 1.5
+    P = torch.softmax(torch.from_numpy(q @ k.T) / math.sqrt(8), dim=1).numpy()
+    for budget in range(1, 11):
+        best = np.array([max(P[t, list(c)].sum() for c in itertools.combinations(range(10), budget))
+                         for t in range(3)])
+        np.testing.assert_allclose(O.token_topk_bound(q, k, budget), best, rtol=0, atol=1e-12)
+
+
+def test_token_bound_closed_forms():
+    rng = np.random.default_rng(72)
+    k = rng.normal(size=(37, 16))
+    # equal logits (q = 0): every token holds 1/n, the bound is budget / n
+    q0 = np.zeros((2, 16))
+    for b in (1, 5, 37):
+        np.testing.assert_allclose(O.token_topk_bound(q0, k, b), b / 37.0, rtol=0, atol=1e-14)
+    # the full budget holds everything
+    q = rng.normal(size=(4, 16))
+    np.testing.assert_allclose(O.token_topk_bound(q, k, 37), 1.0, rtol=0, atol=1e-12)
+    # one key dominating by 60 logits: a single kept token already holds (almost) all of it
+    k2 = k.copy()
+    k2[11] = q[0] * 60.0 * 4.0 / np.dot(q[0], q[0])
+    assert O.token_topk_bound(q[:1], k2, 1)[0] >= 1 - 1e-15 > O.token_topk_bound(q[:1], k, 1)[0]
+
+
+def test_token_bound_dominates_block_mask_and_is_concave():
+    """Any mask with B kept tokens retains at most the bound; the bound grows with B by
+    non-increasing steps (the sorted probabilities); per-row budgets are honoured."""
+    d = 32
+    q = _rand_bf16((256, d), 73).double().numpy()
+    k = _rand_bf16((700, d), 74).double().numpy()
+    v = _rand_bf16((700, d), 75).double().numpy()
+    rows, _ = O.select_head(q, k, 128, 128, 2, 0.5)
+    E, U, R, Ur = O.mass_report(q, k, rows, [0, 1])
+    assert (Ur >= R - 1e-12).all() and (U >= E - 1e-12).all()
+    # R agrees with the LSE form of the retained mass
+    dense = O.dense_attention(q, k, v, [0, 1])
+    kept = O.block_sparse_attention(q, k, v, rows, [0, 1])
+    np.testing.assert_allclose(R, np.concatenate([O.retained_mass(kept[i][1], dense[i][1]) for i in range(2)]),
+                               rtol=0, atol=1e-12)
+    u = np.stack([O.token_topk_bound(q[:5], k, b) for b in range(1, 701)])
+    steps = np.diff(np.vstack([np.zeros((1, 5)), u]), axis=0)
+    assert (steps >= -1e-15).all() and (np.diff(steps, axis=0) <= 1e-15).all()
+    per_row = O.token_topk_bound(q[:3], k, np.array([5, 50, 500]))
+    np.testing.assert_allclose(per_row, [O.token_topk_bound(q[t:t + 1], k, b)[0] for t, b in zip(range(3), (5, 50, 500))],
+                               rtol=0, atol=0)
+    # the ragged last block contributes its valid tokens only
+    assert O.kept_token_count([0, 5], 700) == 128 + 60
