@@ -52,14 +52,15 @@ def parse():
     return ap.parse_args()
 
 
-KERNEL_SOURCES = ("attn_sm100.cuh", "ptx.cuh", "select.cuh", "sparstar.cu")
+ATTN_SOURCES = ("attn_sm100.cuh", "ptx.cuh")   # the attention kernel's device code
 
 
-def kernel_source_hash() -> str:
-    """sha256 (first 16 hex digits) of the CUDA sources the kernels are built from."""
+def kernel_source_hash(sources=ATTN_SOURCES) -> str:
+    """sha256 (first 16 hex digits) of the CUDA sources a kernel is built from (by default the
+    attention kernel's, which keys its DRAM traffic record)."""
     import hashlib
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "block_sparse_attention_tok_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -425,10 +426,11 @@ def run_ours(args, rank, world, local_rank):
         didx = torch.arange(int(dplan.nkb), dtype=torch.int32, device=dev).expand(
             sc.heads, int(dplan.nqb), int(dplan.nkb)).contiguous()
         dcnt = torch.full((sc.heads, int(dplan.nqb)), int(dplan.nkb), dtype=torch.int32, device=dev)
-        S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+        dlse = torch.empty_like(lse)   # lse keeps the sparse step's LSE for the mass analysis
+        S.attn(q, k, v, didx, dcnt, o=o, lse=dlse)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        S.attn(q, k, v, didx, dcnt, o=o, lse=lse)
+        S.attn(q, k, v, didx, dcnt, o=o, lse=dlse)
         e1.record(stream)
         torch.cuda.synchronize()
         dms = e0.elapsed_time(e1)
@@ -436,6 +438,26 @@ def run_ours(args, rank, world, local_rank):
         result["dense"] = {"ms": dms, "tflops": dflops / (dms * 1e-3) / 1e12,
                            "speedup_of_sparse_step": dms / ms}
         del didx, dcnt
+        # Retained dense softmax mass of the selected mask and the token-wise upper bound
+        # with the same per-row token budget (the pages' Figure 3 quantities).
+        S.token_bound(q, k, idx, cnt, dlse, want_tokens=False)   # warm-up
+        m0, m1, m2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        m0.record(stream)
+        _, e_block = S.retained_mass(lse, dlse, want_tokens=False)
+        m1.record(stream)
+        _, u_block = S.token_bound(q, k, idx, cnt, dlse, want_tokens=False)
+        m2.record(stream)
+        torch.cuda.synchronize()
+        bms = m1.elapsed_time(m2)
+        qk_flops = 4 * 2.0 * sc.head_dim * sc.n_q * sc.n_kv * sc.heads   # four dense Q K^T passes
+        result["mass"] = {
+            "retained_mean": float(e_block.mean()), "retained_min": float(e_block.min()),
+            "bound_mean": float(u_block.mean()), "gap_mean": float((u_block - e_block).mean()),
+            "retained_ms": m0.elapsed_time(m1), "bound_ms": bms,
+            "bound_qk_tflops": qk_flops / (bms * 1e-3) / 1e12,
+            "note": "per query block means over valid rows; synthetic inputs, so the pages' values "
+                    "(model activations) are context only"}
+        del dlse, e_block, u_block
 
     # end to end through the public API with host buffers: H2D of q/k/v, forward, D2H of o
     if not args.no_e2e:

@@ -13,7 +13,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libsparstar.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["sparstar.cu"]
-DEPENDS = ["sparstar.cu", "ptx.cuh", "select.cuh", "attn_sm100.cuh"]
+DEPENDS = ["sparstar.cu", "ptx.cuh", "select.cuh", "attn_sm100.cuh", "mass_sm100.cuh"]
 
 
 def nvcc_path() -> str:

@@ -11,6 +11,7 @@
 
 #include "sparstar.h"
 #include "attn_sm100.cuh"
+#include "mass_sm100.cuh"
 #include "select.cuh"
 
 namespace sparstar {
@@ -82,6 +83,10 @@ int set_kernel_attrs(DeviceInfo* d) {
                              AttnConfig<128>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, kPolyCols64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(bound_pass_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BoundConfig<128>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(bound_pass_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BoundConfig<64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ScoreConfig<128>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -369,6 +374,83 @@ int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_
     attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
   else
     attn_sparse_kernel<64, kPolyCols64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+int sparstar_retained_mass(const float* lse_kept, const float* lse_dense, int heads, int64_t n_q, float* r_token,
+                           float* e_block, void* stream) {
+  if (heads < 1 || heads > 65535 || n_q < 0) return SPARSTAR_ERR_ARG;
+  if (n_q == 0) return SPARSTAR_OK;
+  if (lse_kept == nullptr || lse_dense == nullptr || e_block == nullptr) return SPARSTAR_ERR_ARG;
+  const int64_t nqb = ceil_blocks(n_q);
+  if (nqb > INT32_MAX) return SPARSTAR_ERR_UNSUPPORTED;
+  mass_kernel<<<dim3(static_cast<unsigned>(nqb), static_cast<unsigned>(heads)), 128, 0,
+                static_cast<cudaStream_t>(stream)>>>(lse_kept, lse_dense, n_q, static_cast<int>(nqb), r_token, e_block);
+  return launch_status();
+}
+
+int sparstar_token_bound_workspace_size(int heads, int64_t n_q, size_t* bytes) {
+  if (bytes == nullptr || heads < 1 || n_q < 0) return SPARSTAR_ERR_ARG;
+  *bytes = 4 * align256(static_cast<size_t>(heads) * static_cast<size_t>(n_q) * 4);
+  return SPARSTAR_OK;
+}
+
+int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, int64_t n_kv, int head_dim,
+                         const int32_t* idx, const int32_t* cnt, int32_t kmax, const float* lse_dense, float sm_scale,
+                         float* u_token, float* u_block, void* workspace, size_t workspace_bytes, void* stream) {
+  if (heads < 1 || heads > 65535 || n_q < 0 || n_kv < 1 || kmax < 1) return SPARSTAR_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SPARSTAR_ERR_ARG;
+  if (n_q == 0) return SPARSTAR_OK;
+  if (q == nullptr || k == nullptr || idx == nullptr || cnt == nullptr || lse_dense == nullptr ||
+      u_block == nullptr || !aligned16(q) || !aligned16(k))
+    return SPARSTAR_ERR_ARG;
+  size_t need = 0;
+  sparstar_token_bound_workspace_size(heads, n_q, &need);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SPARSTAR_ERR_WORKSPACE;
+  const int64_t nqb = ceil_blocks(n_q), nkb = ceil_blocks(n_kv);
+  if (static_cast<int64_t>(heads) * nqb > INT32_MAX / 2 || n_q > INT32_MAX || n_kv > INT32_MAX || nqb > 65535 * 64LL)
+    return SPARSTAR_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;
+  if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
+  CUtensorMap tq, tk;
+  if (make_map(&tq, q, n_q, heads, head_dim) != SPARSTAR_OK || make_map(&tk, k, n_kv, heads, head_dim) != SPARSTAR_OK)
+    return SPARSTAR_ERR_CUDA;
+  const size_t arr = align256(static_cast<size_t>(heads) * static_cast<size_t>(n_q) * 4);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  BoundParams p;
+  p.st.lo_idx = reinterpret_cast<int*>(w);
+  p.st.need = reinterpret_cast<int*>(w + arr);
+  p.st.above_sum = reinterpret_cast<float*>(w + 2 * arr);
+  p.st.u = reinterpret_cast<float*>(w + 3 * arr);
+  p.lse_dense = lse_dense;
+  p.u_block = u_block;
+  p.status = dev->status;
+  p.n_q = n_q;
+  p.n_kv = n_kv;
+  p.nqb = static_cast<int>(nqb);
+  p.nkb = static_cast<int>(nkb);
+  p.n_items = static_cast<int>(heads * nqb);
+  const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 rows_grid(static_cast<unsigned>(nqb), static_cast<unsigned>(heads));
+  bound_init_kernel<<<rows_grid, 128, 0, st>>>(idx, cnt, kmax, n_q, n_kv, p.nqb, p.st, dev->status);
+  if ((rc = launch_status()) != SPARSTAR_OK) return rc;
+  const int grid = p.n_items < dev->sms ? p.n_items : dev->sms;
+  for (int pass = 0; pass < kBoundPasses; ++pass) {
+    p.pass = pass;
+    if (head_dim == 128)
+      bound_pass_kernel<128><<<grid, BoundConfig<128>::kThreads, BoundConfig<128>::kSmemBytes, st>>>(tq, tk, p);
+    else
+      bound_pass_kernel<64><<<grid, BoundConfig<64>::kThreads, BoundConfig<64>::kSmemBytes, st>>>(tq, tk, p);
+    if ((rc = launch_status()) != SPARSTAR_OK) return rc;
+  }
+  bound_block_kernel<<<rows_grid, 128, 0, st>>>(p.st.u, n_q, p.nqb, u_token, u_block);
   return launch_status();
 }
 

@@ -62,6 +62,14 @@ _SIGNATURES.update({
                                            _c.c_int, _c.c_double, _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32,
                                            _c.c_void_p]),
 })
+_SIGNATURES.update({
+    "sparstar_retained_mass": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, _c.c_void_p, _c.c_void_p,
+                                          _c.c_void_p]),
+    "sparstar_token_bound_workspace_size": (_c.c_int, [_c.c_int, _c.c_int64, _c.POINTER(_c.c_size_t)]),
+    "sparstar_token_bound": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                        _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_float, _c.c_void_p,
+                                        _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+})
 NOALLOC_SCRATCH_BYTES = 128 << 20
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -181,6 +189,46 @@ def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, c
                                 idx.shape[-1], float(sm_scale), _ptr(o), _ptr(lse), _stream_ptr(stream)),
            "sparstar_attn")
     return o, lse
+
+
+def _check_lse(*ts):
+    for t in ts:
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 2:
+            raise ValueError("LSEs must be contiguous fp32 CUDA tensors of shape [H, Nq]")
+
+
+def retained_mass(lse_kept: torch.Tensor, lse_dense: torch.Tensor, want_tokens: bool = True, stream=None):
+    """Retained dense softmax mass of a mask from the two LSEs of sparstar_attn (mask / all
+    blocks). Returns (R fp32 [H,Nq] or None, per-query-block mean fp32 [H,nqb])."""
+    _check_lse(lse_kept, lse_dense)
+    H, n_q = lse_kept.shape
+    nqb = -(-n_q // 128)
+    r = torch.empty(H, n_q, dtype=torch.float32, device=lse_kept.device) if want_tokens else None
+    e = torch.empty(H, nqb, dtype=torch.float32, device=lse_kept.device)
+    _check(load().sparstar_retained_mass(_ptr(lse_kept), _ptr(lse_dense), H, n_q, _ptr(r), _ptr(e),
+                                         _stream_ptr(stream)), "sparstar_retained_mass")
+    return r, e
+
+
+def token_bound(q: torch.Tensor, k: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor, lse_dense: torch.Tensor,
+                sm_scale: float = 0.0, want_tokens: bool = True, stream=None):
+    """Token-wise upper bound on the retained mass with each row's kept-token budget.
+    Returns (U fp32 [H,Nq] or None, per-query-block mean fp32 [H,nqb])."""
+    _check_qkv(q, k)
+    _check_lse(lse_dense)
+    H, n_q, d = q.shape
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous() or not cnt.is_contiguous():
+        raise ValueError("idx/cnt must be contiguous int32")
+    nqb = -(-n_q // 128)
+    nbytes = ctypes.c_size_t()
+    _check(load().sparstar_token_bound_workspace_size(H, n_q, ctypes.byref(nbytes)), "sparstar_token_bound_workspace_size")
+    ws = torch.empty(max(int(nbytes.value), 256), dtype=torch.uint8, device=q.device)
+    u = torch.empty(H, n_q, dtype=torch.float32, device=q.device) if want_tokens else None
+    ub = torch.empty(H, nqb, dtype=torch.float32, device=q.device)
+    _check(load().sparstar_token_bound(_ptr(q), _ptr(k), H, n_q, k.shape[1], d, _ptr(idx), _ptr(cnt), idx.shape[-1],
+                                       _ptr(lse_dense), float(sm_scale), _ptr(u), _ptr(ub), _ptr(ws), int(nbytes.value),
+                                       _stream_ptr(stream)), "sparstar_token_bound")
+    return u, ub
 
 
 def forward(q, k, v, n_text, n_ctx, n_cur, clip, density, budget_mode=BUDGET_LITERAL, sm_scale=0.0,

@@ -157,6 +157,37 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
                             int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
                             void* stream);
 
+/* Retained attention mass of a block mask (digest, 关键结果与论文证据, bullet 跨尺度复用损失,
+ * Figure 3; block energy of eq. (5) of the CalibAtt notes): for every valid query token t,
+ * R_t = exp(lse_kept[t] - lse_dense[t]), the share of its dense softmax mass on the kept
+ * tokens, and per query block the mean of R_t over its valid tokens.
+ * lse_kept / lse_dense: fp32 [H,Nq] device, natural-log LSEs of sparstar_attn with the mask
+ * and with every block kept (cnt = nkb). r_token: fp32 [H,Nq] device or NULL;
+ * e_block: fp32 [H,nqb] device. n_q == 0 is a no-op. */
+int sparstar_retained_mass(const float* lse_kept, const float* lse_dense, int heads,
+                           int64_t n_q, float* r_token, float* e_block, void* stream);
+
+/* Device bytes of the workspace of sparstar_token_bound: four [H,Nq] arrays of 4 bytes. */
+int sparstar_token_bound_workspace_size(int heads, int64_t n_q, size_t* bytes);
+
+/* Token-wise upper bound on the retained mass (same passage): for every valid query token t
+ * of query block i, U_t = the sum of the B_i largest dense softmax probabilities of row t
+ * over all Nkv tokens, B_i = the number of valid KV tokens in the blocks
+ * idx[h][i][0..cnt-1]; per query block the mean of U_t. Computed from the dense logits
+ * sm_scale * q . k (recomputed on the tensor cores, every (query block, KV block) tile, four
+ * times) normalised by lse_dense; the B_i-th largest value is located to 2^-14 in log2 and
+ * the boundary bin's mean stands in for its last values (relative error of U below 5e-5
+ * beyond the logits' own rounding). q [H,Nq,d], k [H,Nkv,d] bf16 device; idx/cnt as for
+ * sparstar_attn (out-of-range entries are skipped and SPARSTAR_ERR_DEVICE_BOUNDS recorded);
+ * lse_dense fp32 [H,Nq] (natural log, from sparstar_attn with every block kept);
+ * sm_scale <= 0 selects 1/sqrt(d). u_token: fp32 [H,Nq] device or NULL; u_block: fp32
+ * [H,nqb] device. workspace: device, >= sparstar_token_bound_workspace_size() bytes,
+ * 256-byte aligned. Requires an sm_100 device. n_q == 0 is a no-op. */
+int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, int64_t n_kv,
+                         int head_dim, const int32_t* idx, const int32_t* cnt, int32_t kmax,
+                         const float* lse_dense, float sm_scale, float* u_token, float* u_block,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then returns SPARSTAR_OK, SPARSTAR_ERR_DEVICE_TIMEOUT or
  * SPARSTAR_ERR_DEVICE_BOUNDS from the current device's status word (timeout wins), or
  * SPARSTAR_ERR_CUDA if the synchronization itself failed. clear != 0 resets the word. */
