@@ -126,49 +126,69 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 template <int D>
 struct ScoreConfig {
   static constexpr int kChunks = D / 64;                    // 128-byte swizzle chunks per row
-  static constexpr uint32_t kQChunk = 128 * 128;            // 128 query-block rows x 128 B
-  static constexpr uint32_t kKChunk = 256 * 128;            // 256 KV-block rows x 128 B
-  static constexpr uint32_t kQBytes = kChunks * kQChunk;    // hi (or lo) tile of qbar
-  static constexpr uint32_t kKBytes = kChunks * kKChunk;    // hi (or lo) tile of kbar
-  static constexpr uint32_t kOperandBytes = 2 * kQBytes + 2 * kKBytes;
-  static constexpr uint32_t kStageRow = 260;                // floats per staged S row (256 + pad)
-  static constexpr uint32_t kStageBytes = 128 * kStageRow * 4;
-  // Operands and the epilogue's staging area share one region (used one after the other).
-  static constexpr uint32_t kDataBytes = kOperandBytes > kStageBytes ? kOperandBytes : kStageBytes;
-  static constexpr uint32_t kSmemBytes = 1024 + kDataBytes + 64;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);
-  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kChunkBytes = 128 * 128;        // 128 rows x 128 B
+  static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;  // hi (or lo) of 128 block means
+  static constexpr int kStages = 2;                         // K (hi + lo) ring
+  static constexpr int kThreads = 192;                      // TMA warp, MMA warp, 4 epilogue warps
+  static constexpr int kStageRow = 65;                      // floats per staged row (64 + pad)
+  static constexpr uint32_t kStageBytes = 4 * 32 * kStageRow * 4;   // per epilogue warp: 32 rows x 64
+  static constexpr uint32_t kSmemBytes = 1024 + 2 * kTileBytes + kStages * 2 * kTileBytes + kStageBytes + 256;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
+  static constexpr uint32_t kTmemCols = 256;                // two 128-column accumulators
 };
 
-// grid = (ceil(nkb/256), ceil(nqb/128), H); 128 threads. One elected thread loads the four
-// tiles with TMA (out-of-range rows are zero) and issues 3 * D/16 MMAs of M=128, N=256, K=16;
-// each warp then reads its 32 rows of the fp32 accumulator and writes S.
+// S = qbar kbar^T / sqrt(d) for every (head, 128 query blocks, 128 KV blocks) tile, as
+// hi.hi + hi.lo + lo.hi bf16 products (fp32 accumulation in tensor memory). Persistent: CTA c
+// takes a contiguous run of tiles in (head, query tile, KV tile) order, so consecutive tiles
+// share the query tile, which stays in shared memory; KV tiles stream through a two-stage
+// TMA ring while the previous tile's epilogue (tensor memory -> registers -> a padded staging
+// buffer -> coalesced rows of S) runs on the other accumulator. Out-of-range rows load as
+// zero and are not stored.
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(ScoreConfig<D>::kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_ql,
                     const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kl,
-                    float* __restrict__ S, int nqb, int nkb, float inv_sqrt_d, unsigned* status) {
+                    float* __restrict__ S, int heads, int nqb, int nkb, float inv_sqrt_d, unsigned* status) {
   using C = ScoreConfig<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* qh_s = smem;
-  uint8_t* ql_s = qh_s + C::kQBytes;
-  uint8_t* kh_s = ql_s + C::kQBytes;
-  uint8_t* kl_s = kh_s + C::kKBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kDataBytes);
-  uint64_t* done = full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint8_t* q_s = smem;                                // [hi | lo]
+  uint8_t* k_s = smem + 2 * C::kTileBytes;            // [stage][hi | lo]
+  float* stage_buf = reinterpret_cast<float*>(k_s + C::kStages * 2 * C::kTileBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage_buf) + C::kStageBytes);
+  uint64_t* full = bars;                  // [kStages]
+  uint64_t* empty = full + C::kStages;    // [kStages]
+  uint64_t* q_full = empty + C::kStages;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* acc_full = q_empty + 1;       // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2], 128 arrivals
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.z, i0 = blockIdx.y * 128, j0 = blockIdx.x * 256;
+
+  const int n_mt = (nqb + 127) / 128, n_nt = (nkb + 127) / 128;
+  const int n_tiles = heads * n_mt * n_nt;
+  const int per_cta = (n_tiles + gridDim.x - 1) / gridDim.x;
+  const int t_begin = blockIdx.x * per_cta;
+  const int t_end = min(n_tiles, t_begin + per_cta);
 
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
-    mbar_init(done, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -179,73 +199,149 @@ __global__ void __launch_bounds__(128, 1)
   griddep_launch_dependents();
   griddep_wait();  // pooled means come from the preceding pool kernel
 
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(full, 2 * C::kQBytes + 2 * C::kKBytes);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int q_key = -1, q_loads = 0;
+      uint32_t ring_it = 0;
+      for (int t = t_begin; t < t_end; ++t) {
+        const int nt = t % n_nt, hm = t / n_nt, mt = hm % n_mt, h = hm / n_mt;
+        if (hm != q_key) {  // a new query tile: once the MMAs of the previous one are done
+          if (!mbar_wait(q_empty, (q_loads & 1) ^ 1, abort_flag, status)) break;
+          mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
 #pragma unroll
-    for (int c = 0; c < C::kChunks; ++c) {
-      tma_load_3d(smem_u32(qh_s + c * C::kQChunk), &tm_qh, full, c * 64, i0, h);
-      tma_load_3d(smem_u32(ql_s + c * C::kQChunk), &tm_ql, full, c * 64, i0, h);
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_3d(smem_u32(q_s) + c * C::kChunkBytes, &tm_qh, q_full, c * 64, mt * 128, h);
+            tma_load_3d(smem_u32(q_s) + C::kTileBytes + c * C::kChunkBytes, &tm_ql, q_full, c * 64, mt * 128, h);
+          }
+          q_key = hm;
+          ++q_loads;
+        }
+        const uint32_t st = ring_it % C::kStages;
+        if (!mbar_wait(&empty[st], ((ring_it / C::kStages) & 1u) ^ 1u, abort_flag, status)) break;
+        mbar_arrive_expect_tx(&full[st], 2 * C::kTileBytes);
+        const uint32_t dst = smem_u32(k_s) + st * 2 * C::kTileBytes;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tma_load_3d(smem_u32(kh_s + c * C::kKChunk + half * 16384), &tm_kh, full, c * 64, j0 + 128 * half, h);
-        tma_load_3d(smem_u32(kl_s + c * C::kKChunk + half * 16384), &tm_kl, full, c * 64, j0 + 128 * half, h);
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(dst + c * C::kChunkBytes, &tm_kh, &full[st], c * 64, nt * 128, h);
+          tma_load_3d(dst + C::kTileBytes + c * C::kChunkBytes, &tm_kl, &full[st], c * 64, nt * 128, h);
+        }
+        ++ring_it;
       }
-    }
-    if (mbar_wait(full, 0, abort_flag, status)) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t qa = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
-        const uint32_t kb = (kk >> 2) * C::kKChunk + (kk & 3) * 32;
-        const uint64_t dqh = smem_desc_sw128(smem_u32(qh_s) + qa, 16, 1024);
-        const uint64_t dql = smem_desc_sw128(smem_u32(ql_s) + qa, 16, 1024);
-        const uint64_t dkh = smem_desc_sw128(smem_u32(kh_s) + kb, 16, 1024);
-        const uint64_t dkl = smem_desc_sw128(smem_u32(kl_s) + kb, 16, 1024);
-        mma_ss(tmem, dqh, dkh, C::kIdesc, kk > 0 ? 1u : 0u);
-        mma_ss(tmem, dqh, dkl, C::kIdesc, 1u);
-        mma_ss(tmem, dql, dkh, C::kIdesc, 1u);
+      // Drain: every issued load lands before the CTA exits (matters only after an abort).
+      for (uint32_t s2 = 0; s2 < C::kStages; ++s2) {
+        if (ring_it > s2) {
+          const uint32_t last_use = ring_it - 1 - ((ring_it - 1 - s2) % C::kStages);
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[s2], (last_use / C::kStages) & 1u) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
       }
-    }
-    mma_commit(done);  // also arrives when nothing was issued
-  }
-  __syncwarp();
-  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag, status));
-  tc_fence_after();
-  if (ok) {
-    // Stage this warp's 32 rows x 256 columns in the (now idle) operand buffers, padded to
-    // 260 floats per row so that the 16-byte stores of 32 rows hit distinct banks, then
-    // write whole row segments with coalesced stores.
-    float* stage = reinterpret_cast<float*>(smem) + warp * 32 * C::kStageRow;
-    float* my_row = stage + lane * C::kStageRow;
-#pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32 * c, r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(my_row + 32 * c + e) =
-            make_float4(__uint_as_float(r[e]) * inv_sqrt_d, __uint_as_float(r[e + 1]) * inv_sqrt_d,
-                        __uint_as_float(r[e + 2]) * inv_sqrt_d, __uint_as_float(r[e + 3]) * inv_sqrt_d);
+      if (q_loads > 0) {
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, (q_loads - 1) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
     }
     __syncwarp();
-    const int n_cols = min(256, nkb - j0);
-#pragma unroll 1
-    for (int rr = 0; rr < 32; ++rr) {
-      const int i = i0 + warp * 32 + rr;
-      if (i >= nqb) break;
-      float* srow = S + (static_cast<int64_t>(h) * nqb + i) * nkb + j0;
-      const float* src = stage + rr * C::kStageRow;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (whole warp, elected lane)
+    const uint64_t qh_d = smem_desc_sw128(smem_u32(q_s), 16, 1024);
+    const uint64_t ql_d = qh_d + (C::kTileBytes >> 4);
+    const uint64_t k_d = smem_desc_sw128(smem_u32(k_s), 16, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, status));
+    };
+    int q_key = -1, q_loads = 0;
+    uint32_t ring_it = 0, acc_it = 0;
+    for (int t = t_begin; t < t_end; ++t, ++acc_it) {
+      const int hm = t / n_nt;
+      if (hm != q_key) {
+        if (!wait_all(q_full, q_loads & 1)) break;
+        q_key = hm;
+        ++q_loads;
+      }
+      const uint32_t a = acc_it & 1u;
+      if (acc_it >= 2 && !wait_all(&acc_empty[a], ((acc_it >> 1) - 1) & 1u)) break;
+      const uint32_t st = ring_it % C::kStages;
+      if (!wait_all(&full[st], (ring_it / C::kStages) & 1u)) break;
+      tc_fence_after();
+      const uint64_t kh_d = k_d + ((st * 2 * C::kTileBytes) >> 4);
+      const uint64_t kl_d = kh_d + (C::kTileBytes >> 4);
+      const bool last_of_q = (t + 1 == t_end) || ((t + 1) / n_nt != hm);
+      if (elect_one()) {
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const int col = lane + 32 * cc;
-        if (col < n_cols) srow[col] = src[col];
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + 128u * a, qh_d + off, kh_d + off, C::kIdesc, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + 128u * a, qh_d + off, kl_d + off, C::kIdesc, 1u);
+          mma_ss(tmem + 128u * a, ql_d + off, kh_d + off, C::kIdesc, 1u);
+        }
+        mma_commit(&empty[st]);
+        mma_commit(&acc_full[a]);
+        if (last_of_q) mma_commit(q_empty);
+      }
+      __syncwarp();
+      ++ring_it;
+    }
+    if (elect_one()) mma_commit(drain);
+    __syncwarp();
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    const int wq = warp & 3;                 // TMEM lane quarter: rows 32*wq .. 32*wq + 31
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    float* stg = stage_buf + (warp - 2) * 32 * C::kStageRow;
+    uint32_t acc_it = 0;
+    for (int t = t_begin; t < t_end; ++t, ++acc_it) {
+      const int nt = t % n_nt, hm = t / n_nt, mt = hm % n_mt, h = hm / n_mt;
+      const uint32_t a = acc_it & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[a], (acc_it >> 1) & 1u, abort_flag, status))) break;
+      tc_fence_after();
+      const int j0 = nt * 128;
+      const int n_cols = min(128, nkb - j0);
+      const int i_base = mt * 128 + wq * 32;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[2][32];
+        tmem_ld32(tmem + lane_off + 128u * a + 64u * half, r[0]);
+        tmem_ld32(tmem + lane_off + 128u * a + 64u * half + 32u, r[1]);
+        tmem_wait_ld();
+        if (half == 1) {  // the accumulator is in registers: the MMA may reuse it
+          tc_fence_before();
+          mbar_arrive(&acc_empty[a]);
+        }
+        // lane = row: stage this warp's 32 rows x 64 columns (row stride 65 floats, so both
+        // the row-wise writes here and the column-wise reads below hit 32 distinct banks)
+        float* my_row = stg + lane * C::kStageRow;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) my_row[32 * c + e] = __uint_as_float(r[c][e]) * inv_sqrt_d;
+        __syncwarp();
+        const int col0 = 64 * half;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr) {
+          const int i = i_base + rr;
+          if (i >= nqb) break;
+          float* srow = S + (static_cast<int64_t>(h) * nqb + i) * nkb + j0 + col0;
+          const float* src = stg + rr * C::kStageRow;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int col = lane + 32 * cc;
+            if (col0 + col < n_cols) srow[col] = src[col];
+          }
+        }
+        __syncwarp();
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -404,7 +500,7 @@ __global__ void __launch_bounds__(128) fill_kernel(int k_total, int32_t* __restr
 template <int KPL>
 __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, int n_forced, int n_cand, int k_topk,
                                               int32_t* __restrict__ out, uint32_t* gather, uint32_t* hist,
-                                              float* sv, uint16_t* lst) {
+                                              float* sv, uint16_t* lst, uint8_t* bins) {
   const int lane = threadIdx.x & 31;
   const uint32_t full = 0xFFFFFFFFu;
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -442,14 +538,23 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, in
   const float width = smax - smin;
   const float scale = width > 0.f ? 256.f / width : 0.f;
   const float offset = -smin * scale;
-  auto bin_of = [&](float x) -> uint32_t {  // monotone in x; NaN -> 0
+  // Bin of a score: f = (x - min) * 256 / width in [0, 256], rounded to nearest by adding
+  // 1.5 * 2^23 (the integer lands in the low mantissa bits), clamped to 255; monotone in x,
+  // NaN -> 0. Computed once per candidate and kept in shared memory.
+  auto bin_of = [&](float x) -> uint32_t {
     const float f = fmaf(x, scale, offset);
-    return f != f ? 0u : min(255u, __float2uint_rz(f));
+    return f != f ? 0u : min(255u, __float_as_uint(f + 12582912.0f) & 0x3FFu);
   };
   // 2. histogram and the bin of the K-th largest key
 #pragma unroll
-  for (int t = 0; t < KPL; ++t)
-    if (lane + 32 * t < n_cand) atomicAdd(&hist[bin_of(sv[lane + 32 * t])], 1u);
+  for (int t = 0; t < KPL; ++t) {
+    const int j = lane + 32 * t;
+    if (j < n_cand) {
+      const uint32_t b = bin_of(sv[j]);
+      bins[j] = static_cast<uint8_t>(b);
+      atomicAdd(&hist[b], 1u);
+    }
+  }
   __syncwarp();
   uint32_t cnt[8], local = 0;  // lane l owns bins 255-8l .. 248-8l (descending)
 #pragma unroll
@@ -488,7 +593,7 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, in
 #pragma unroll
   for (int t = 0; t < KPL; ++t) {
     const int j = lane + 32 * t;
-    const bool in = j < n_cand && bin_of(sv[j]) >= bstar;
+    const bool in = j < n_cand && bins[j] >= bstar;
     const uint32_t ball = __ballot_sync(full, in);
     if (in) lst[m + __popc(ball & lt_mask)] = static_cast<uint16_t>(j);
     m += __popc(ball);
@@ -497,9 +602,9 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, in
   // 4. key range of b*, narrowed while it holds more than 32 keys
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
   for (uint32_t e = lane; e < m; e += 32) {
-    const float x = sv[lst[e]];
-    if (bin_of(x) == bstar) {
-      const uint32_t k = key_of(x);
+    const uint32_t j = lst[e];
+    if (bins[j] == bstar) {
+      const uint32_t k = key_of(sv[j]);
       kmin = min(kmin, k);
       kmax = max(kmax, k);
     }
@@ -570,7 +675,8 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, in
 
 template <int KPL>
 constexpr int topk_warp_smem() {
-  return 8 * 32 * KPL * (4 + 2);  // per warp: scores (fp32) and the compacted index list (uint16)
+  // per warp: scores (fp32), the compacted index list (uint16) and the score bins (uint8)
+  return 8 * 32 * KPL * (4 + 2 + 1);
 }
 
 // One warp per row, 8 rows per 256-thread CTA; grid.x = ceil(H * nqb / 8). Requires
@@ -587,8 +693,9 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict_
   griddep_wait();  // scores come from the preceding score kernel
   if (row >= rows) return;
   uint16_t* lists = reinterpret_cast<uint16_t*>(rowbuf + 8 * 32 * KPL);
+  uint8_t* bins = reinterpret_cast<uint8_t*>(lists + 8 * 32 * KPL);
   topk_row_warp<KPL>(S + row * nkb, n_forced, nkb - n_forced, k_topk, idx + row * kmax, gather[w], hist[w],
-                     rowbuf + w * 32 * KPL, lists + w * 32 * KPL);
+                     rowbuf + w * 32 * KPL, lists + w * 32 * KPL, bins + w * 32 * KPL);
   if ((threadIdx.x & 31) == 0) cnt[row] = n_forced + k_topk;
 }
 

@@ -283,20 +283,21 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
         make_map(&tkl, k_lo, nkb, heads, head_dim) != SPARSTAR_OK)
       return SPARSTAR_ERR_CUDA;
     const unsigned pool_grid = static_cast<unsigned>(heads) * static_cast<unsigned>(nqb + nkb);
-    const dim3 sgrid((nkb + 255) / 256, (nqb + 127) / 128, heads);
+    const int score_tiles = heads * ((nqb + 127) / 128) * ((nkb + 127) / 128);
+    const dim3 sgrid(static_cast<unsigned>(score_tiles < dev->sms ? score_tiles : dev->sms));
     const float inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(head_dim));
     if (head_dim == 128) {
       pool_kernel<128><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                   static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
                                                   q_lo, k_hi, k_lo);
-      launch_after(score_tc_kernel<128>, sgrid, dim3(128), ScoreConfig<128>::kSmemBytes, st, tqh, tql, tkh, tkl, S, nqb,
-                   nkb, inv_sqrt_d, dev->status);
+      launch_after(score_tc_kernel<128>, sgrid, dim3(ScoreConfig<128>::kThreads), ScoreConfig<128>::kSmemBytes, st, tqh,
+                   tql, tkh, tkl, S, heads, nqb, nkb, inv_sqrt_d, dev->status);
     } else {
       pool_kernel<64><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
                                                  q_lo, k_hi, k_lo);
-      launch_after(score_tc_kernel<64>, sgrid, dim3(128), ScoreConfig<64>::kSmemBytes, st, tqh, tql, tkh, tkl, S, nqb,
-                   nkb, inv_sqrt_d, dev->status);
+      launch_after(score_tc_kernel<64>, sgrid, dim3(ScoreConfig<64>::kThreads), ScoreConfig<64>::kSmemBytes, st, tqh,
+                   tql, tkh, tkl, S, heads, nqb, nkb, inv_sqrt_d, dev->status);
     }
     if ((rc = launch_status()) != SPARSTAR_OK) return rc;
     if (needs_scores) {
