@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-block64", action="store_true", help="skip the 64-token block variant")
     ap.add_argument("--no-schedule", action="store_true",
                     help="skip the per-scale timing of the refined-scale schedule (4 scales x 36 layers)")
     return ap.parse_args()
@@ -149,16 +150,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- accounting
 
-def kept_tile_flops(idx: torch.Tensor, cnt: torch.Tensor, n_q: int, n_kv: int, d: int) -> float:
+def kept_tile_flops(idx: torch.Tensor, cnt: torch.Tensor, n_q: int, n_kv: int, d: int, block: int = 128) -> float:
     """4 d * sum over kept tiles of valid_query_rows * valid_kv_tokens (bookkeeping only)."""
     H, nqb, kmax = idx.shape
     col = torch.arange(kmax, device=idx.device)
     live = col[None, None, :] < cnt[:, :, None]
-    nkb = -(-n_kv // 128)
-    vk = torch.where(idx == nkb - 1, n_kv - (nkb - 1) * 128, 128).to(torch.float64)
+    nkb = -(-n_kv // block)
+    vk = torch.where(idx == nkb - 1, n_kv - (nkb - 1) * block, block).to(torch.float64)
     per_row = (vk * live).sum(-1)
-    vq = torch.full((nqb,), 128.0, dtype=torch.float64, device=idx.device)
-    vq[-1] = n_q - (nqb - 1) * 128
+    vq = torch.full((nqb,), float(block), dtype=torch.float64, device=idx.device)
+    vq[-1] = n_q - (nqb - 1) * block
     return float(4.0 * d * (per_row * vq[None, :]).sum().item())
 
 
@@ -419,6 +420,42 @@ def run_ours(args, rank, world, local_rank):
     }
     clocks_summary = clocks.summary()
     result["clocks"] = clocks_summary
+
+    # The 64-token block variant on the same input (the pages' block-size ablation): same path,
+    # block = 64 for the partition, the scores, the Top-K and the attention tiles.
+    if not args.no_block64 and not args.heads:
+        plan64 = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode, block=64)
+        ws64 = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev, block=64)
+        idx64 = torch.empty(sc.heads, int(plan64.nqb), int(plan64.k_total), dtype=torch.int32, device=dev)
+        cnt64 = torch.empty(sc.heads, int(plan64.nqb), dtype=torch.int32, device=dev)
+        o64 = torch.empty_like(q)
+
+        def step64(ev):
+            ev[0].record(stream)
+            S.select(q, k, *seg, sc.clip, sc.density, args.budget_mode, workspace=ws64, idx=idx64, cnt=cnt64, block=64)
+            ev[1].record(stream)
+            S.attn(q, k, v, idx64, cnt64, o=o64, want_lse=False, block=64)
+            ev[2].record(stream)
+
+        n64 = max(3, min(args.steps, 5))
+        ev64 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n64 + 2)]
+        for e in ev64:
+            step64(e)
+        torch.cuda.synchronize()
+        t_sel64 = float(np.median([e[0].elapsed_time(e[1]) for e in ev64[2:]]))
+        t_att64 = float(np.median([e[1].elapsed_time(e[2]) for e in ev64[2:]]))
+        flops64 = kept_tile_flops(idx64, cnt64, sc.n_q, sc.n_kv, sc.head_dim, block=64)
+        sel_bytes64 = 2.0 * sc.heads * sc.head_dim * (sc.n_q + sc.n_kv) + 4.0 * sc.heads * plan64.nqb * (plan64.k_total + 1)
+        result["block64"] = {
+            "nqb": int(plan64.nqb), "nkb": int(plan64.nkb), "k_total": int(plan64.k_total),
+            "k_topk": int(plan64.k_topk), "n_cand": int(plan64.n_cand),
+            "attn_ms": t_att64, "attn_tflops": flops64 / (t_att64 * 1e-3) / 1e12,
+            "kept_tile_tflop": flops64 / 1e12, "select_us": t_sel64 * 1e3,
+            "select_gbs": sel_bytes64 / (t_sel64 * 1e-3) / 1e9, "step_ms": t_sel64 + t_att64,
+            "note": "64-row query blocks run as half of a 128-row MMA tile and 64-token KV tiles use "
+                    "N = 64 MMAs, so per kept FLOP the tensor cores do about 2x the work of block 128"}
+        del ws64, idx64, cnt64, o64
+        torch.cuda.empty_cache()
 
     # dense run of the same shape: the same kernel with every block kept
     if not args.no_dense:

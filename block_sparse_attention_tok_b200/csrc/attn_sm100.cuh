@@ -35,15 +35,22 @@
 
 namespace sparstar {
 
-template <int D>
+// B = block size of the partition (128, or 64 for the block-size variant): a query block is B
+// rows of the 128-row MMA tile (with B = 64 the other 64 rows are computed and dropped) and a
+// KV tile is one B-token KV block (MMA N = B for QK^T, K = B for PV).
+template <int D, int B = 128>
 struct AttnConfig {
   static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
-  static constexpr int kRows = 128;                    // query rows per tile (one query block)
-  static constexpr int kCols = 128;                    // KV tokens per tile (one KV block)
+  static_assert(B == 64 || B == 128, "block must be 64 or 128");
+  static constexpr int kRows = 128;                    // query rows per MMA tile
+  static constexpr int kCols = B;                      // KV tokens per tile (one KV block)
+  static constexpr int kSC = B / 32;                   // 32-column chunks of an S row
   static constexpr int kChunks = D / 64;               // 128-byte swizzle chunks per row
-  static constexpr uint32_t kChunkBytes = 128 * 128;   // 128 rows x 128 bytes
-  static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring depth
+  static constexpr uint32_t kQChunkBytes = 128 * 128;  // 128 rows x 128 bytes
+  static constexpr uint32_t kKVChunkBytes = B * 128;   // B rows x 128 bytes
+  static constexpr uint32_t kQTileBytes = kChunks * kQChunkBytes;
+  static constexpr uint32_t kKVTileBytes = kChunks * kKVChunkBytes;
+  static constexpr int kStages = ((D == 128) ? 4 : 8) * (128 / B);  // K/V ring depth
   static constexpr int kSlots = 2;
   static constexpr int kThreads = 320;                 // 8 softmax warps + TMA warp + MMA warp
   static constexpr int kLoadWarp = 8;
@@ -51,8 +58,8 @@ struct AttnConfig {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS = 0;                // + 128 * slot
   static constexpr uint32_t kTmemO = 256;              // + 128 * slot
-  static constexpr uint32_t kSmemBytes = 1024 /*align*/ + kSlots * kTileBytes + kStages * kTileBytes + 512;
-  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
+  static constexpr uint32_t kSmemBytes = 1024 /*align*/ + kSlots * kQTileBytes + kStages * kKVTileBytes + 512;
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, B, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
 };
 
@@ -131,19 +138,24 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Max of a 128-column S row held as four 32-register chunks: 8 independent 3-input max
-// chains, then a short tree (dependency depth 10 instead of 128).
-__device__ __forceinline__ float row_max128(const uint32_t (&r)[4][32]) {
+// Max of a (32*NC)-column S row held as NC 32-register chunks: 8 independent chains, chain i
+// covering column i of every group of 8 columns (3-input max over two groups per step), then
+// a short tree (dependency depth 11 instead of 128 for NC = 4).
+template <int NC>
+__device__ __forceinline__ float row_max(const uint32_t (&r)[NC][32]) {
+  constexpr int G = 4 * NC;  // groups of 8 columns
+  auto col = [&](int c) { return __uint_as_float(r[c >> 5][c & 31]); };
   float m[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m[i] = fmax3(__uint_as_float(r[0][i]), __uint_as_float(r[0][i + 8]), __uint_as_float(r[0][i + 16]));
+  for (int i = 0; i < 8; ++i) m[i] = col(i);
 #pragma unroll
-  for (int k = 24; k < 128; k += 16)
+  for (int g = 1; g + 1 < G; g += 2)
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      m[i] = fmax3(m[i], __uint_as_float(r[(k + i) >> 5][(k + i) & 31]),
-                   __uint_as_float(r[(k + 8 + i) >> 5][(k + 8 + i) & 31]));
+    for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], col(8 * g + i), col(8 * g + 8 + i));
+  if ((G - 1) % 2 == 1) {  // the last group has no partner
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], col(8 * (G - 1) + i));
+  }
   return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
@@ -167,19 +179,19 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-template <int D, int kPolyCols>
-__global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
+template <int D, int kPolyCols, int B = 128>
+__global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     attn_sparse_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using C = AttnConfig<D>;
-  static_assert(kPolyCols % 32 == 0 && kPolyCols <= 128, "software exp2 works on whole 32-column chunks");
+  using C = AttnConfig<D, B>;
+  static_assert(kPolyCols % 32 == 0 && kPolyCols <= B, "software exp2 works on whole 32-column chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint8_t* q_tile = smem;                                   // [slot] kTileBytes each
-  uint8_t* ring = smem + C::kSlots * C::kTileBytes;         // [stage] kTileBytes each
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::kStages * C::kTileBytes);
+  uint8_t* q_tile = smem;                                   // [slot] kQTileBytes each
+  uint8_t* ring = smem + C::kSlots * C::kQTileBytes;        // [stage] kKVTileBytes each
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::kStages * C::kKVTileBytes);
   uint64_t* full = bars;                      // [kStages] TMA -> MMA
   uint64_t* empty = full + C::kStages;        // [kStages] MMA -> TMA
   uint64_t* q_full = empty + C::kStages;      // [2]
@@ -237,11 +249,11 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
 
       auto load_q = [&](int s, SlotSeq& sq, int& last_k) -> bool {
         if (!mbar_wait(&q_empty[s], (sq.k & 1) ^ 1, abort_flag, p.status)) return false;
-        mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
-        const uint32_t dst = smem_u32(q_tile + s * C::kTileBytes);
+        mbar_arrive_expect_tx(&q_full[s], C::kQTileBytes);
+        const uint32_t dst = smem_u32(q_tile + s * C::kQTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kChunkBytes, &tm_q, &q_full[s], c * 64, sq.qb * 128, sq.h);
+          tma_load_3d(dst + c * C::kQChunkBytes, &tm_q, &q_full[s], c * 64, sq.qb * B, sq.h);
         last_k = sq.k;
         return true;
       };
@@ -250,11 +262,11 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         const uint32_t stage = ring_it % C::kStages;
         const uint32_t phase = (ring_it / C::kStages) & 1u;
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
-        mbar_arrive_expect_tx(&full[stage], C::kTileBytes);
-        const uint32_t dst = smem_u32(ring + stage * C::kTileBytes);
+        mbar_arrive_expect_tx(&full[stage], C::kKVTileBytes);
+        const uint32_t dst = smem_u32(ring + stage * C::kKVTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kChunkBytes, map, &full[stage], c * 64, j * 128, sq.h);
+          tma_load_3d(dst + c * C::kKVChunkBytes, map, &full[stage], c * 64, j * B, sq.h);
         ++ring_it;
         return true;
       };
@@ -310,7 +322,7 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
     // 2^18, so desc(addr + off) = desc(addr) + (off >> 4) for 16-byte multiples off.
     const uint64_t q_desc = smem_desc_sw128(smem_u32(q_tile), 16, 1024);
     const uint64_t k_desc = smem_desc_sw128(smem_u32(ring), 16, 1024);
-    const uint64_t v_desc = smem_desc_sw128(smem_u32(ring), C::kChunkBytes, 1024);
+    const uint64_t v_desc = smem_desc_sw128(smem_u32(ring), C::kKVChunkBytes, 1024);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, p.status));
     };
@@ -321,14 +333,15 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
       if (sq.n == 0 && !wait_all(&q_full[s], sq.k & 1)) return false;
       const uint32_t stage = ring_it % C::kStages;
       if (!wait_all(&full[stage], (ring_it / C::kStages) & 1u)) return false;
-      const uint64_t qd = q_desc + ((s * C::kTileBytes) >> 4);
-      const uint64_t kd = k_desc + ((stage * C::kTileBytes) >> 4);
+      const uint64_t qd = q_desc + ((s * C::kQTileBytes) >> 4);
+      const uint64_t kd = k_desc + ((stage * C::kKVTileBytes) >> 4);
       const uint32_t d_tmem = tmem_base + C::kTmemS + 128u * s;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
-          mma_ss(d_tmem, qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t qoff = ((kk >> 2) * C::kQChunkBytes + (kk & 3) * 32) >> 4;
+          const uint32_t koff = ((kk >> 2) * C::kKVChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, qd + qoff, kd + koff, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
         mma_commit(&s_full[s]);
@@ -344,15 +357,15 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
       const uint32_t stage = ring_it % C::kStages;
       if (!wait_all(&full[stage], (ring_it / C::kStages) & 1u)) return false;
       tc_fence_after();  // P was written by the softmax warps with tcgen05.st
-      const uint64_t vd = v_desc + ((stage * C::kTileBytes) >> 4);
+      const uint64_t vd = v_desc + ((stage * C::kKVTileBytes) >> 4);
       const uint32_t d_tmem = tmem_base + C::kTmemO + 128u * s;
       const uint32_t a_tmem = tmem_base + C::kTmemS + 128u * s;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < B / 16; ++kk) {
           // P columns: 16 bf16 per K step = 8 packed 32-bit columns.
-          // V tile is MN-major for this MMA: 64-element chunks of d at 16 KB (LBO), 8-row
-          // groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
+          // V tile is MN-major for this MMA: 64-element chunks of d at B*128 bytes (LBO),
+          // 8-row groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
           mma_ts(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), C::kIdescPV, (sq.n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
@@ -403,7 +416,7 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
       for (int n = 0; n < seq.ntiles && ok; ++n) {
         seq.n = n;
         const int j = seq_block(seq, p, false);
-        const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * 128) : 128;
+        const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * B) : B;
         // tcgen05.ld/st below are warp-collective: every lane must take the same path.
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], tiles & 1u, abort_flag, p.status))) {
           ok = false;
@@ -411,18 +424,18 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         }
         ++tiles;
         tc_fence_after();
-        uint32_t r[4][32];
+        uint32_t r[C::kSC][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r[c]);
+        for (int c = 0; c < C::kSC; ++c) tmem_ld32(t_s + 32 * c, r[c]);
         tmem_wait_ld();
-        if (n_valid < 128) {
+        if (n_valid < B) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < C::kSC; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               if (32 * c + e >= n_valid) r[c][e] = __float_as_uint(-INFINITY);
         }
-        const float mx_scaled = row_max128(r) * p.scale_log2;
+        const float mx_scaled = row_max<C::kSC>(r) * p.scale_log2;
         float alpha = 1.f;
         if (mx_scaled > m_run + 8.f) {
           alpha = ex2_approx(m_run - mx_scaled);  // m_run = -inf on the first tile -> 0
@@ -436,14 +449,14 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < C::kSC; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[c][2 * e]), __uint_as_float(r[c][2 * e + 1])),
                                         scale2, neg_m2);
             float2 pr;
-            if (c >= 4 - kPolyCols / 32) {
+            if (c >= C::kSC - kPolyCols / 32) {
               pr = exp2_poly2(x);
             } else {
               pr.x = ex2_approx(x.x);
@@ -469,9 +482,9 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
             tmem_st32(t_o + 32 * c, ov);
           }
         }
-        // P: 128 bf16 = 64 packed columns over the start of S.
+        // P: B bf16 = B/2 packed columns over the start of S.
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < C::kSC / 2; ++c) {
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -489,8 +502,8 @@ __global__ void __launch_bounds__(AttnConfig<D>::kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_full[s], items & 1u, abort_flag, p.status))) break;
       ++items;
       tc_fence_after();
-      const int64_t t = static_cast<int64_t>(seq.qb) * 128 + row;
-      const bool valid = t < p.n_q;
+      const int64_t t = static_cast<int64_t>(seq.qb) * B + row;
+      const bool valid = row < B && t < p.n_q;  // with B = 64, rows 64-127 belong to the next block
       const float inv_l = 1.f / l_run;
       __nv_bfloat16* orow = p.o + (static_cast<int64_t>(seq.h) * p.n_q + t) * D;
 #pragma unroll 1

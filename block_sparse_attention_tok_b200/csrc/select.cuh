@@ -3,19 +3,22 @@
 // Follows the SparSTAR digest ("SparSTAR的贡献：每尺度动态重建", pchao.org), section 方法概览:
 // Q and KV are cut into 128-token blocks, each block is mean-pooled, every (query block,
 // key block) pair gets an aggregate score from the pooled vectors, the clip-aware forced
-// blocks are kept, and the rest of each row is filled by a joint Top-K, per head.
+// blocks are kept, and the rest of each row is filled by a joint Top-K, per head. The block
+// size is a template parameter (128, or 64 for the block-size variant of the pages'
+// ablation, section 实验如何设计?, bullet on supplementary experiments).
 //
 // Kernels:
-//   pool_kernel      one CTA per 128-token block: 16-byte streaming loads, fp32 sums,
-//                    shuffle + shared-memory reduction, divide by the valid token count; the
-//                    mean m is stored as two bf16 numbers hi = bf16(m), lo = bf16(m - hi).
-//   score_tc_kernel  S = qbar kbar^T / sqrt(d) on the tensor cores: per CTA a 128 x 256 tile
-//                    of (query block, KV block) pairs, TMA-fed, tcgen05.mma accumulating
-//                    hi.hi + hi.lo + lo.hi in fp32 tensor memory (the dropped lo.lo term and
-//                    the bf16 rounding of lo keep the error near 2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
-//   topk_warp_kernel one warp per (head, query block) row, keys in registers: the K-th largest
-//                    key is bracketed by counting, then resolved among <= 32 keys by a warp
-//                    bitonic sort; ties taken lowest index first, ascending emit.
+//   pool_kernel      one CTA per block: 16-byte streaming loads, fp32 sums, shuffle +
+//                    shared-memory reduction, divide by the valid token count; the mean m is
+//                    stored as two bf16 numbers hi = bf16(m), lo = bf16(m - hi).
+//   score_tc_kernel  S = qbar kbar^T / sqrt(d) on the tensor cores: persistent CTAs over
+//                    128 x 128 tiles of (query block, KV block) pairs, TMA-fed,
+//                    tcgen05.mma accumulating hi.hi + hi.lo + lo.hi in fp32 tensor memory
+//                    (the dropped lo.lo term and the bf16 rounding of lo keep the error near
+//                    2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
+//   topk_warp_kernel one warp per (head, query block) row: the K-th largest key is bracketed
+//                    by a value histogram, then resolved among <= 32 keys by a warp bitonic
+//                    sort; ties taken lowest index first, ascending emit.
 //   topk_kernel      one CTA per row, 8-bit radix select in shared memory (rows with more than
 //                    2048 candidates).
 //   fill_kernel      rows that do not depend on scores (K_topk == 0 or every block kept):
@@ -50,7 +53,7 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
 
 // grid.x = H * (nq_blocks + nk_blocks) (Q blocks of a head first, then its K blocks);
 // nq_blocks may be 0 (pool K only). 256 threads. Outputs [H, n_blocks, D] bf16 hi and lo.
-template <int D>
+template <int D, int B = 128>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, int64_t n_q,
                                                    int64_t n_kv, int nq_blocks, int nk_blocks,
@@ -58,7 +61,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    __nv_bfloat16* __restrict__ k_hi, __nv_bfloat16* __restrict__ k_lo) {
   constexpr int kChunks = D / 8;           // 16-byte chunks per token row
   constexpr int kRowGroups = 256 / kChunks;
-  constexpr int kRowsPerThread = 128 / kRowGroups;
+  constexpr int kRowsPerThread = B / kRowGroups;  // B = tokens per block (128, or 64)
   __shared__ float part[8][D];
   griddep_launch_dependents();  // the score kernel may be scheduled early; it waits for this grid
 
@@ -84,8 +87,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     dst_hi = k_hi + o;
     dst_lo = k_lo + o;
   }
-  const int64_t row0 = b * 128;
-  const int n_valid = static_cast<int>(min(static_cast<int64_t>(128), n_tok - row0));
+  const int64_t row0 = b * B;
+  const int n_valid = static_cast<int>(min(static_cast<int64_t>(B), n_tok - row0));
   const int c = threadIdx.x % kChunks;
   const int rg = threadIdx.x / kChunks;
 

@@ -83,6 +83,10 @@ int set_kernel_attrs(DeviceInfo* d) {
                              AttnConfig<128>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, kPolyCols64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128, 0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnConfig<128, 64>::kSmemBytes) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, 0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnConfig<64, 64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(bound_pass_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BoundConfig<128>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(bound_pass_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -104,7 +108,8 @@ int set_kernel_attrs(DeviceInfo* d) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int64_t ceil_blocks(int64_t n) { return (n + SPARSTAR_BLOCK - 1) / SPARSTAR_BLOCK; }
+int64_t ceil_blocks(int64_t n, int64_t block = SPARSTAR_BLOCK) { return (n + block - 1) / block; }
+bool valid_block(int block) { return block == 64 || block == 128; }
 
 // ceil(x) with a 1e-9 guard, so that a product such as 0.1875 * 16 = 3.0 stays 3.
 int64_t ceil_guarded(double x) { return static_cast<int64_t>(std::ceil(x - 1e-9)); }
@@ -162,11 +167,11 @@ int topk_keys_per_lane(int64_t n_cand) {
   return 0;
 }
 
-int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d) {
-  // 3-D view [heads][rows][d] of bf16; box = 64 elements x 128 rows x 1 head, 128B swizzle.
+int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, unsigned box_rows = 128) {
+  // 3-D view [heads][rows][d] of bf16; box = 64 elements x box_rows rows x 1 head, 128B swizzle.
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -197,18 +202,19 @@ const char* sparstar_strerror(int code) {
   }
 }
 
-int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double density, int budget_mode,
-                       sparstar_plan* out) {
+int sparstar_make_plan_ex(int64_t n_q, sparstar_segments seg, int clip, double density, int budget_mode, int block,
+                          sparstar_plan* out) {
   if (out == nullptr || n_q < 0 || !valid_segments(seg) || clip < 1 || !(density > 0.0) || !(density <= 1.0) ||
       (budget_mode != SPARSTAR_BUDGET_LITERAL && budget_mode != SPARSTAR_BUDGET_CANDIDATES))
     return SPARSTAR_ERR_ARG;
+  if (!valid_block(block)) return SPARSTAR_ERR_UNSUPPORTED;
   const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
   if (n_kv < 1) return SPARSTAR_ERR_ARG;
   sparstar_plan p;
-  p.nqb = ceil_blocks(n_q);
-  p.nkb = ceil_blocks(n_kv);
+  p.nqb = ceil_blocks(n_q, block);
+  p.nkb = ceil_blocks(n_kv, block);
   const int64_t forced_tokens = seg.n_text + (clip == 1 ? seg.n_ctx : 0);
-  p.n_forced = ceil_blocks(forced_tokens);
+  p.n_forced = ceil_blocks(forced_tokens, block);
   if (p.n_forced > p.nkb) p.n_forced = p.nkb;
   p.n_cand = p.nkb - p.n_forced;
   int64_t k_total, k_topk;
@@ -230,20 +236,30 @@ int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double dens
   return SPARSTAR_OK;
 }
 
-int sparstar_workspace_size(int heads, int64_t n_q, sparstar_segments seg, int head_dim, size_t* bytes) {
+int sparstar_make_plan(int64_t n_q, sparstar_segments seg, int clip, double density, int budget_mode,
+                       sparstar_plan* out) {
+  return sparstar_make_plan_ex(n_q, seg, clip, density, budget_mode, SPARSTAR_BLOCK, out);
+}
+
+int sparstar_workspace_size_ex(int heads, int64_t n_q, sparstar_segments seg, int head_dim, int block, size_t* bytes) {
   if (bytes == nullptr || heads < 1 || n_q < 0 || !valid_segments(seg)) return SPARSTAR_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  if (!valid_block(block)) return SPARSTAR_ERR_UNSUPPORTED;
   const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
   if (n_kv < 1) return SPARSTAR_ERR_ARG;
-  *bytes = workspace_layout(heads, ceil_blocks(n_q), ceil_blocks(n_kv), head_dim, true).total;
+  *bytes = workspace_layout(heads, ceil_blocks(n_q, block), ceil_blocks(n_kv, block), head_dim, true).total;
   return SPARSTAR_OK;
 }
 
-int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparstar_segments seg, int head_dim,
-                    int clip, double density, int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
-                    float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+int sparstar_workspace_size(int heads, int64_t n_q, sparstar_segments seg, int head_dim, size_t* bytes) {
+  return sparstar_workspace_size_ex(heads, n_q, seg, head_dim, SPARSTAR_BLOCK, bytes);
+}
+
+int sparstar_select_ex(const void* q, const void* k, int heads, int64_t n_q, sparstar_segments seg, int head_dim,
+                       int clip, double density, int budget_mode, int block, int32_t* idx, int32_t* cnt, int32_t kmax,
+                       float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   sparstar_plan plan;
-  int rc = sparstar_make_plan(n_q, seg, clip, density, budget_mode, &plan);
+  int rc = sparstar_make_plan_ex(n_q, seg, clip, density, budget_mode, block, &plan);
   if (rc != SPARSTAR_OK) return rc;
   if (heads < 1) return SPARSTAR_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
@@ -286,16 +302,20 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
     const int score_tiles = heads * ((nqb + 127) / 128) * ((nkb + 127) / 128);
     const dim3 sgrid(static_cast<unsigned>(score_tiles < dev->sms ? score_tiles : dev->sms));
     const float inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(head_dim));
+    const auto* qb16 = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb16 = static_cast<const __nv_bfloat16*>(k);
     if (head_dim == 128) {
-      pool_kernel<128><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                  static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
-                                                  q_lo, k_hi, k_lo);
+      if (block == 128)
+        pool_kernel<128, 128><<<pool_grid, 256, 0, st>>>(qb16, kb16, n_q, n_kv, nqb, nkb, q_hi, q_lo, k_hi, k_lo);
+      else
+        pool_kernel<128, 64><<<pool_grid, 256, 0, st>>>(qb16, kb16, n_q, n_kv, nqb, nkb, q_hi, q_lo, k_hi, k_lo);
       launch_after(score_tc_kernel<128>, sgrid, dim3(ScoreConfig<128>::kThreads), ScoreConfig<128>::kSmemBytes, st, tqh,
                    tql, tkh, tkl, S, heads, nqb, nkb, inv_sqrt_d, dev->status);
     } else {
-      pool_kernel<64><<<pool_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                 static_cast<const __nv_bfloat16*>(k), n_q, n_kv, nqb, nkb, q_hi,
-                                                 q_lo, k_hi, k_lo);
+      if (block == 128)
+        pool_kernel<64, 128><<<pool_grid, 256, 0, st>>>(qb16, kb16, n_q, n_kv, nqb, nkb, q_hi, q_lo, k_hi, k_lo);
+      else
+        pool_kernel<64, 64><<<pool_grid, 256, 0, st>>>(qb16, kb16, n_q, n_kv, nqb, nkb, q_hi, q_lo, k_hi, k_lo);
       launch_after(score_tc_kernel<64>, sgrid, dim3(ScoreConfig<64>::kThreads), ScoreConfig<64>::kSmemBytes, st, tqh,
                    tql, tkh, tkl, S, heads, nqb, nkb, inv_sqrt_d, dev->status);
     }
@@ -331,18 +351,26 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
   return launch_status();
 }
 
-int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_t n_q, int64_t n_kv, int head_dim,
-                  const int32_t* idx, const int32_t* cnt, int32_t kmax, float sm_scale, void* o, float* lse,
-                  void* stream) {
+int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparstar_segments seg, int head_dim,
+                    int clip, double density, int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
+                    float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+  return sparstar_select_ex(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, SPARSTAR_BLOCK, idx, cnt,
+                            kmax, scores, workspace, workspace_bytes, stream);
+}
+
+int sparstar_attn_ex(const void* q, const void* k, const void* v, int heads, int64_t n_q, int64_t n_kv, int head_dim,
+                     int block, const int32_t* idx, const int32_t* cnt, int32_t kmax, float sm_scale, void* o,
+                     float* lse, void* stream) {
   if (heads < 1 || n_q < 0 || n_kv < 1 || kmax < 1) return SPARSTAR_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return SPARSTAR_ERR_UNSUPPORTED;
+  if (!valid_block(block)) return SPARSTAR_ERR_UNSUPPORTED;
   if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SPARSTAR_ERR_ARG;
   if (n_q == 0) return SPARSTAR_OK;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || idx == nullptr || cnt == nullptr ||
       !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
     return SPARSTAR_ERR_ARG;
-  const int64_t nqb = ceil_blocks(n_q), nkb = ceil_blocks(n_kv);
+  const int64_t nqb = ceil_blocks(n_q, block), nkb = ceil_blocks(n_kv, block);
   if (static_cast<int64_t>(heads) * nqb > INT32_MAX / 2 || n_q > INT32_MAX || n_kv > INT32_MAX || nkb > INT32_MAX)
     return SPARSTAR_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
@@ -351,8 +379,10 @@ int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_
   if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;
   if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
   CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, n_q, heads, head_dim) != SPARSTAR_OK || make_map(&tk, k, n_kv, heads, head_dim) != SPARSTAR_OK ||
-      make_map(&tv, v, n_kv, heads, head_dim) != SPARSTAR_OK)
+  const unsigned kv_rows = static_cast<unsigned>(block);
+  if (make_map(&tq, q, n_q, heads, head_dim) != SPARSTAR_OK ||
+      make_map(&tk, k, n_kv, heads, head_dim, kv_rows) != SPARSTAR_OK ||
+      make_map(&tv, v, n_kv, heads, head_dim, kv_rows) != SPARSTAR_OK)
     return SPARSTAR_ERR_CUDA;
   AttnParams p;
   p.idx = idx;
@@ -371,11 +401,24 @@ int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int slots_needed = (p.n_items + 1) / 2;
   const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
-  if (head_dim == 128)
-    attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
-  else
-    attn_sparse_kernel<64, kPolyCols64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+  if (block == 128) {
+    if (head_dim == 128)
+      attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
+    else
+      attn_sparse_kernel<64, kPolyCols64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+  } else {
+    if (head_dim == 128)
+      attn_sparse_kernel<128, 0, 64><<<grid, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
+    else
+      attn_sparse_kernel<64, 0, 64><<<grid, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
+  }
   return launch_status();
+}
+
+int sparstar_attn(const void* q, const void* k, const void* v, int heads, int64_t n_q, int64_t n_kv, int head_dim,
+                  const int32_t* idx, const int32_t* cnt, int32_t kmax, float sm_scale, void* o, float* lse,
+                  void* stream) {
+  return sparstar_attn_ex(q, k, v, heads, n_q, n_kv, head_dim, SPARSTAR_BLOCK, idx, cnt, kmax, sm_scale, o, lse, stream);
 }
 
 int sparstar_retained_mass(const float* lse_kept, const float* lse_dense, int heads, int64_t n_q, float* r_token,
@@ -455,15 +498,23 @@ int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, i
   return launch_status();
 }
 
+int sparstar_forward_ex(const void* q, const void* k, const void* v, int heads, int64_t n_q, sparstar_segments seg,
+                        int head_dim, int clip, double density, int budget_mode, int block, float sm_scale,
+                        int32_t* idx, int32_t* cnt, int32_t kmax, void* o, float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  int rc = sparstar_select_ex(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, block, idx, cnt, kmax,
+                              nullptr, workspace, workspace_bytes, stream);
+  if (rc != SPARSTAR_OK) return rc;
+  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
+  return sparstar_attn_ex(q, k, v, heads, n_q, n_kv, head_dim, block, idx, cnt, kmax, sm_scale, o, lse, stream);
+}
+
 int sparstar_forward(const void* q, const void* k, const void* v, int heads, int64_t n_q, sparstar_segments seg,
                      int head_dim, int clip, double density, int budget_mode, float sm_scale, int32_t* idx,
                      int32_t* cnt, int32_t kmax, void* o, float* lse, void* workspace, size_t workspace_bytes,
                      void* stream) {
-  int rc = sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
-                           workspace, workspace_bytes, stream);
-  if (rc != SPARSTAR_OK) return rc;
-  const int64_t n_kv = seg.n_text + seg.n_ctx + seg.n_cur;
-  return sparstar_attn(q, k, v, heads, n_q, n_kv, head_dim, idx, cnt, kmax, sm_scale, o, lse, stream);
+  return sparstar_forward_ex(q, k, v, heads, n_q, seg, head_dim, clip, density, budget_mode, SPARSTAR_BLOCK, sm_scale,
+                             idx, cnt, kmax, o, lse, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- no-allocation selection

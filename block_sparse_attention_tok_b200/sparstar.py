@@ -58,6 +58,20 @@ _SIGNATURES.update({
                                     _c.c_int, _c.c_double, _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p,
                                     _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "sparstar_device_status": (_c.c_int, [_c.c_void_p, _c.c_int]),
+    "sparstar_make_plan_ex": (_c.c_int, [_c.c_int64, Segments, _c.c_int, _c.c_double, _c.c_int, _c.c_int,
+                                         _c.POINTER(Plan)]),
+    "sparstar_workspace_size_ex": (_c.c_int, [_c.c_int, _c.c_int64, Segments, _c.c_int, _c.c_int,
+                                              _c.POINTER(_c.c_size_t)]),
+    "sparstar_select_ex": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments, _c.c_int, _c.c_int,
+                                      _c.c_double, _c.c_int, _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32,
+                                      _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "sparstar_attn_ex": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                    _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_float, _c.c_void_p,
+                                    _c.c_void_p, _c.c_void_p]),
+    "sparstar_forward_ex": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments,
+                                       _c.c_int, _c.c_int, _c.c_double, _c.c_int, _c.c_int, _c.c_float, _c.c_void_p,
+                                       _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
+                                       _c.c_void_p]),
     "sparstar_select_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, Segments, _c.c_int,
                                            _c.c_int, _c.c_double, _c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32,
                                            _c.c_void_p]),
@@ -122,17 +136,18 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def make_plan(n_q: int, n_text: int, n_ctx: int, n_cur: int, clip: int, density: float,
-              budget_mode: int = BUDGET_LITERAL) -> Plan:
+              budget_mode: int = BUDGET_LITERAL, block: int = BLOCK) -> Plan:
     plan = Plan()
-    _check(load().sparstar_make_plan(int(n_q), Segments(n_text, n_ctx, n_cur), int(clip), float(density),
-                                     int(budget_mode), ctypes.byref(plan)), "sparstar_make_plan")
+    _check(load().sparstar_make_plan_ex(int(n_q), Segments(n_text, n_ctx, n_cur), int(clip), float(density),
+                                        int(budget_mode), int(block), ctypes.byref(plan)), "sparstar_make_plan_ex")
     return plan
 
 
-def workspace_size(heads: int, n_q: int, n_text: int, n_ctx: int, n_cur: int, head_dim: int) -> int:
+def workspace_size(heads: int, n_q: int, n_text: int, n_ctx: int, n_cur: int, head_dim: int,
+                   block: int = BLOCK) -> int:
     out = ctypes.c_size_t()
-    _check(load().sparstar_workspace_size(int(heads), int(n_q), Segments(n_text, n_ctx, n_cur), int(head_dim),
-                                          ctypes.byref(out)), "sparstar_workspace_size")
+    _check(load().sparstar_workspace_size_ex(int(heads), int(n_q), Segments(n_text, n_ctx, n_cur), int(head_dim),
+                                             int(block), ctypes.byref(out)), "sparstar_workspace_size_ex")
     return int(out.value)
 
 
@@ -145,19 +160,21 @@ def _check_qkv(*ts):
 class Workspace:
     """Reusable device workspace sized for one shape (allocated once by torch)."""
 
-    def __init__(self, heads, n_q, n_text, n_ctx, n_cur, head_dim, device):
-        nbytes = workspace_size(heads, n_q, n_text, n_ctx, n_cur, head_dim)
+    def __init__(self, heads, n_q, n_text, n_ctx, n_cur, head_dim, device, block: int = 128):
+        nbytes = workspace_size(heads, n_q, n_text, n_ctx, n_cur, head_dim, block)
         self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         self.nbytes = nbytes
 
 
 def select(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_cur: int, clip: int, density: float,
            budget_mode: int = BUDGET_LITERAL, want_scores: bool = False, workspace: Optional[Workspace] = None,
-           idx: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None, stream=None):
-    """Block selection. Returns (idx [H,nqb,K_total] int32, cnt [H,nqb] int32, scores or None)."""
+           idx: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None, stream=None,
+           block: int = BLOCK):
+    """Block selection with `block`-token blocks (128, or 64). Returns (idx [H,nqb,K_total]
+    int32, cnt [H,nqb] int32, scores or None)."""
     _check_qkv(q, k)
     H, n_q, d = q.shape
-    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode)
+    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode, block)
     nqb, nkb, kmax = int(plan.nqb), int(plan.nkb), max(int(plan.k_total), 1)
     if idx is None:
         idx = torch.empty(H, nqb, kmax, dtype=torch.int32, device=q.device)
@@ -165,18 +182,19 @@ def select(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_cur: int
         cnt = torch.empty(H, nqb, dtype=torch.int32, device=q.device)
     scores = torch.empty(H, nqb, nkb, dtype=torch.float32, device=q.device) if want_scores else None
     if workspace is None:
-        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device)
-    _check(load().sparstar_select(_ptr(q), _ptr(k), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
-                                  float(density), int(budget_mode), _ptr(idx), _ptr(cnt), idx.shape[-1],
-                                  _ptr(scores), _ptr(workspace.buf), workspace.nbytes, _stream_ptr(stream)),
-           "sparstar_select")
+        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device, block)
+    _check(load().sparstar_select_ex(_ptr(q), _ptr(k), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
+                                     float(density), int(budget_mode), int(block), _ptr(idx), _ptr(cnt),
+                                     idx.shape[-1], _ptr(scores), _ptr(workspace.buf), workspace.nbytes,
+                                     _stream_ptr(stream)), "sparstar_select_ex")
     return idx, cnt, scores
 
 
 def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor,
          sm_scale: float = 0.0, o: Optional[torch.Tensor] = None, want_lse: bool = True,
-         lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Block-sparse attention over the kept tiles. Returns (o bf16 [H,Nq,d], lse fp32 [H,Nq] or None)."""
+         lse: Optional[torch.Tensor] = None, stream=None, block: int = BLOCK) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Block-sparse attention over the kept tiles (`block`-token blocks). Returns (o bf16
+    [H,Nq,d], lse fp32 [H,Nq] or None)."""
     _check_qkv(q, k, v)
     H, n_q, d = q.shape
     if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous() or not cnt.is_contiguous():
@@ -185,9 +203,9 @@ def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, c
         o = torch.empty_like(q)
     if want_lse and lse is None:
         lse = torch.empty(H, n_q, dtype=torch.float32, device=q.device)
-    _check(load().sparstar_attn(_ptr(q), _ptr(k), _ptr(v), H, n_q, k.shape[1], d, _ptr(idx), _ptr(cnt),
-                                idx.shape[-1], float(sm_scale), _ptr(o), _ptr(lse), _stream_ptr(stream)),
-           "sparstar_attn")
+    _check(load().sparstar_attn_ex(_ptr(q), _ptr(k), _ptr(v), H, n_q, k.shape[1], d, int(block), _ptr(idx),
+                                   _ptr(cnt), idx.shape[-1], float(sm_scale), _ptr(o), _ptr(lse), _stream_ptr(stream)),
+           "sparstar_attn_ex")
     return o, lse
 
 
@@ -233,11 +251,11 @@ def token_bound(q: torch.Tensor, k: torch.Tensor, idx: torch.Tensor, cnt: torch.
 
 def forward(q, k, v, n_text, n_ctx, n_cur, clip, density, budget_mode=BUDGET_LITERAL, sm_scale=0.0,
             workspace: Optional[Workspace] = None, idx=None, cnt=None, o=None, lse=None, want_lse=True,
-            stream=None):
+            stream=None, block: int = BLOCK):
     """The whole per-scale path (selection then attention). Returns (o, lse, idx, cnt)."""
     _check_qkv(q, k, v)
     H, n_q, d = q.shape
-    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode)
+    plan = make_plan(n_q, n_text, n_ctx, n_cur, clip, density, budget_mode, block)
     kmax = max(int(plan.k_total), 1)
     if idx is None:
         idx = torch.empty(H, int(plan.nqb), kmax, dtype=torch.int32, device=q.device)
@@ -248,11 +266,11 @@ def forward(q, k, v, n_text, n_ctx, n_cur, clip, density, budget_mode=BUDGET_LIT
     if want_lse and lse is None:
         lse = torch.empty(H, n_q, dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device)
-    _check(load().sparstar_forward(_ptr(q), _ptr(k), _ptr(v), H, n_q, Segments(n_text, n_ctx, n_cur), d, int(clip),
-                                   float(density), int(budget_mode), float(sm_scale), _ptr(idx), _ptr(cnt),
-                                   idx.shape[-1], _ptr(o), _ptr(lse), _ptr(workspace.buf), workspace.nbytes,
-                                   _stream_ptr(stream)), "sparstar_forward")
+        workspace = Workspace(H, n_q, n_text, n_ctx, n_cur, d, q.device, block)
+    _check(load().sparstar_forward_ex(_ptr(q), _ptr(k), _ptr(v), H, n_q, Segments(n_text, n_ctx, n_cur), d,
+                                      int(clip), float(density), int(budget_mode), int(block), float(sm_scale),
+                                      _ptr(idx), _ptr(cnt), idx.shape[-1], _ptr(o), _ptr(lse), _ptr(workspace.buf),
+                                      workspace.nbytes, _stream_ptr(stream)), "sparstar_forward_ex")
     return o, lse, idx, cnt
 
 

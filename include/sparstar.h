@@ -157,6 +157,31 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
                             int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
                             void* stream);
 
+/* Block-size variants (the pages' block-size ablation, section 实验如何设计?, bullet on the
+ * supplementary experiments): the same calls with the block size of the partition as an
+ * argument, block in {64, 128} (anything else: SPARSTAR_ERR_UNSUPPORTED). Every count in the
+ * plan (nqb, nkb, n_forced, budgets) and every index in idx is then in units of `block`
+ * tokens; a ragged last block holds the remaining tokens. The functions without the suffix
+ * are these with block = SPARSTAR_BLOCK (128). The no-allocation entry point, the retained
+ * mass and the token-wise bound work on 128-token blocks only. */
+int sparstar_make_plan_ex(int64_t n_q, sparstar_segments seg, int clip, double density,
+                          int budget_mode, int block, sparstar_plan* out);
+int sparstar_workspace_size_ex(int heads, int64_t n_q, sparstar_segments seg, int head_dim,
+                               int block, size_t* bytes);
+int sparstar_select_ex(const void* q, const void* k, int heads, int64_t n_q,
+                       sparstar_segments seg, int head_dim, int clip, double density,
+                       int budget_mode, int block, int32_t* idx, int32_t* cnt, int32_t kmax,
+                       float* scores, void* workspace, size_t workspace_bytes, void* stream);
+int sparstar_attn_ex(const void* q, const void* k, const void* v, int heads, int64_t n_q,
+                     int64_t n_kv, int head_dim, int block, const int32_t* idx,
+                     const int32_t* cnt, int32_t kmax, float sm_scale, void* o, float* lse,
+                     void* stream);
+int sparstar_forward_ex(const void* q, const void* k, const void* v, int heads, int64_t n_q,
+                        sparstar_segments seg, int head_dim, int clip, double density,
+                        int budget_mode, int block, float sm_scale, int32_t* idx, int32_t* cnt,
+                        int32_t kmax, void* o, float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
 /* Retained attention mass of a block mask (digest, 关键结果与论文证据, bullet 跨尺度复用损失,
  * Figure 3; block energy of eq. (5) of the CalibAtt notes): for every valid query token t,
  * R_t = exp(lse_kept[t] - lse_dense[t]), the share of its dense softmax mass on the kept

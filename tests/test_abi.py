@@ -8,7 +8,7 @@ import re
 import numpy as np
 import pytest
 
-from block_sparse_attention_tok_b200 import sparstar, _build
+from block_sparse_attention_tok_b200 import sparstar, synth, _build
 from oracle import sparstar_oracle as O
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sparstar.h")
@@ -114,3 +114,18 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_build, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         sparstar.load()
+
+
+def test_block_size_plans_match_oracle_and_reject_other_sizes(lib):
+    from block_sparse_attention_tok_b200 import sparstar as S
+    for sc in (synth.TINY_CLIP2, synth.MID_CLIP1, synth.FINAL_CLIP1_RAGGED, synth.FINAL_CLIP2):
+        for mode in (0, 1):
+            p = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode, block=64)
+            nkb = O.num_blocks(sc.n_kv, 64)
+            nf = min(O.forced_block_count(sc.n_text, sc.n_ctx, sc.clip, 64), nkb)
+            kt, kk = O.row_budget(nkb, nf, sc.density, mode)
+            assert (int(p.nqb), int(p.nkb), int(p.n_forced), int(p.k_total), int(p.k_topk)) == \
+                (O.num_blocks(sc.n_q, 64), nkb, nf, kt, kk)
+    with pytest.raises(S.SparstarError) as e:
+        S.make_plan(1024, 256, 768, 1024, 2, 0.25, 0, block=96)
+    assert e.value.code == S.ERR_UNSUPPORTED

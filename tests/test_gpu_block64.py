@@ -1,0 +1,117 @@
+"""The 64-token block variant (the pages' block-size ablation) on the GPU, against the oracle
+run with block = 64: masks by the same gap rule, outputs element by element.
+
+With 64-token blocks a query block is 64 rows of the kernel's 128-row MMA tile (the other
+64 rows are computed and dropped), a KV tile is one 64-token block, and rows with more than
+2048 candidates go through the radix Top-K.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_tok_b200 import synth
+from oracle import sparstar_oracle as O
+from tests.parity import bits, check_masks, check_output, LSE_ABS
+
+pytestmark = pytest.mark.gpu
+B = 64
+
+
+@pytest.fixture(scope="module")
+def S(cuda_lib):
+    from block_sparse_attention_tok_b200 import sparstar
+    return sparstar
+
+
+def _f64(x):
+    return O.bf16_bits_to_f64(x)
+
+
+def _run(S, q, k, v, n_text, n_ctx, n_cur, clip, density, mode=0, qblocks=None, heads=None):
+    H, n_q, d = q.shape
+    heads = list(range(H)) if heads is None else heads
+    o, lse, idx, cnt = S.forward(q, k, v, n_text, n_ctx, n_cur, clip, density, mode, block=B)
+    _, _, scores = S.select(q, k, n_text, n_ctx, n_cur, clip, density, mode, want_scores=True, block=B)
+    assert S.device_status() == S.OK
+    plan = S.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode, block=B)
+    sel = torch.tensor(heads, device=q.device)
+    qb, kb, vb = bits(q[sel]), bits(k[sel]), bits(v[sel])
+    ref = [O.select_head(_f64(qb[i]), _f64(kb[i]), n_text, n_ctx, clip, density, mode, block=B)
+           for i in range(len(heads))]
+    ref_idx, ref_S = np.stack([r[0] for r in ref]), np.stack([r[1] for r in ref])
+    gidx, gcnt = idx[sel].cpu().numpy(), cnt[sel].cpu().numpy()
+    stats = check_masks(gidx, gcnt, ref_idx, ref_S, int(plan.n_forced), int(plan.k_topk))
+    got_S = scores[sel].cpu().numpy()
+    for hi in range(len(heads)):
+        qbar, kbar = O.pool_blocks(_f64(qb[hi]), B), O.pool_blocks(_f64(kb[hi]), B)
+        bound = 2.0 ** -14 * (np.abs(qbar) @ np.abs(kbar).T) / math.sqrt(d) + 1e-7
+        assert (np.abs(got_S[hi] - ref_S[hi]) <= bound).all()
+    o_np, lse_np = o[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
+    nqb = int(plan.nqb)
+    for hi in range(len(heads)):
+        qbl = range(nqb) if qblocks is None else qblocks(nqb)
+        qbl = [i for i in qbl if (gidx[hi, i, :ref_idx.shape[2]] == ref_idx[hi, i]).all()]
+        outs = O.block_sparse_attention(_f64(qb[hi]), _f64(kb[hi]), _f64(vb[hi]), ref_idx[hi], qbl, block=B)
+        for i, (o_ref, lse_ref) in zip(qbl, outs):
+            s, e = O.block_token_range(i, n_q, B)
+            check_output(o_np[hi, s:e], o_ref, f"h{heads[hi]} qb{i}")
+            assert np.abs(lse_np[hi, s:e] - lse_ref).max() <= LSE_ABS
+    return stats, plan
+
+
+@pytest.mark.parametrize("d,n_q,n_text,n_ctx,n_cur,clip,density", [
+    (64, 300, 128, 256, 300, 2, 0.3),        # ragged query and KV tails (300 = 4*64 + 44)
+    (128, 1000, 256, 1000, 1000, 2, 0.2),
+    (128, 130, 64, 200, 130, 1, 0.5),        # Clip 1: text + context forced; a 2-row last block
+])
+def test_block64_small_cases(S, d, n_q, n_text, n_ctx, n_cur, clip, density):
+    q, k, v = synth.make_qkv(n_q, n_text + n_ctx + n_cur, 2, d, [700 + n_q, 701 + n_q], device="cuda")
+    stats, plan = _run(S, q, k, v, n_text, n_ctx, n_cur, clip, density)
+    assert stats["rows"] == 2 * int(plan.nqb)
+
+
+def test_block64_radix_topk_rows(S):
+    """More than 2048 candidates per row: the CTA-per-row radix Top-K path."""
+    n_cur = 64 * 2100
+    q, k, v = synth.make_qkv(200, 64 + n_cur, 1, 128, [811], device="cuda")
+    stats, plan = _run(S, q, k, v, 64, 0, n_cur, 2, 0.05, qblocks=lambda n: [0, n - 1])
+    assert int(plan.n_cand) > 2048 and stats["rows"] == int(plan.nqb)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n_q,n_kv", [(1, 1), (63, 65), (200, 1000)])
+def test_block64_attention_on_random_masks(S, d, n_q, n_kv):
+    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [17, 18], device="cuda")
+    nqb, nkb = O.num_blocks(n_q, B), O.num_blocks(n_kv, B)
+    rng = np.random.default_rng(n_q * 7 + n_kv)
+    kk = max(1, min(nkb, int(rng.integers(1, nkb + 1))))
+    rows = np.stack([np.stack([np.sort(rng.choice(nkb, kk, replace=False)) for _ in range(nqb)]) for _ in range(2)])
+    idx = torch.from_numpy(rows.astype(np.int32)).cuda().contiguous()
+    cnt = torch.full((2, nqb), kk, dtype=torch.int32, device="cuda")
+    o, lse = S.attn(q, k, v, idx, cnt, block=B)
+    assert S.device_status() == S.OK
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(2):
+        outs = O.block_sparse_attention(_f64(qb[h]), _f64(kb[h]), _f64(vb[h]), rows[h], range(nqb), block=B)
+        for i, (o_ref, lse_ref) in enumerate(outs):
+            s, e = O.block_token_range(i, n_q, B)
+            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
+            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+
+
+@pytest.mark.slow
+def test_block64_final_scale_sampled(S):
+    """The 720p Clip-2 final scale with 64-token blocks (every mask row of 3 heads checked,
+    outputs on sampled query blocks)."""
+    sc = synth.FINAL_CLIP2
+    q, k, v = synth.make_scale_inputs(sc, device="cuda")
+    rng = np.random.default_rng(64)
+    stats, plan = _run(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density,
+                       qblocks=lambda n: sorted({0, n - 1, *rng.choice(n, 3, replace=False).tolist()}),
+                       heads=[0, 15, 31])
+    print(stats)
+    del q, k, v
+    torch.cuda.empty_cache()

@@ -361,3 +361,24 @@ def test_token_bound_dominates_block_mask_and_is_concave():
                                rtol=0, atol=0)
     # the ragged last block contributes its valid tokens only
     assert O.kept_token_count([0, 5], 700) == 128 + 60
+
+
+def test_block_size_consistency_64_vs_128():
+    """The oracle is generic in the block size: a 128-token mask written as 64-token blocks
+    (each kept 128-block -> its two halves) gives the same attention, and a 128-block mean is
+    the mean of its two 64-block means (full blocks)."""
+    d = 32
+    q = _rand_bf16((256, d), 81).double().numpy()
+    k = _rand_bf16((640, d), 82).double().numpy()
+    v = _rand_bf16((640, d), 83).double().numpy()
+    rows128 = np.array([[0, 2, 4], [1, 3, 4]])
+    out128 = O.block_sparse_attention(q, k, v, rows128, [0, 1], block=128)
+    rows64 = np.array([sorted({2 * j + h for j in r for h in (0, 1)}) for r in rows128])
+    rows64 = np.repeat(rows64, 2, axis=0)                  # query blocks 2i, 2i+1 share row i
+    out64 = O.block_sparse_attention(q, k, v, rows64, [0, 1, 2, 3], block=64)
+    for i in range(2):
+        np.testing.assert_allclose(np.vstack([out64[2 * i][0], out64[2 * i + 1][0]]), out128[i][0], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(np.concatenate([out64[2 * i][1], out64[2 * i + 1][1]]), out128[i][1], rtol=0, atol=1e-13)
+    p64, p128 = O.pool_blocks(k, 64), O.pool_blocks(k, 128)
+    np.testing.assert_allclose((p64[0::2] + p64[1::2]) / 2, p128, rtol=0, atol=1e-15)
+    assert O.forced_block_count(512, 8192, 1, 64) == 2 * O.forced_block_count(512, 8192, 1, 128) == 136
