@@ -129,3 +129,15 @@ def test_block_size_plans_match_oracle_and_reject_other_sizes(lib):
     with pytest.raises(S.SparstarError) as e:
         S.make_plan(1024, 256, 768, 1024, 2, 0.25, 0, block=96)
     assert e.value.code == S.ERR_UNSUPPORTED
+
+
+def test_select_rejects_more_candidates_than_supported_before_launch(lib):
+    """n_cand = 16,385 is one past the radix Top-K's shared-memory limit: refused before any
+    device call (fake device addresses are never touched)."""
+    n_kv = 128 * (1 + 16385)
+    rc = lib.sparstar_select(0x1000, 0x2000, 1, 256, sparstar.Segments(128, 0, n_kv - 128), 64, 2, 0.05, 0,
+                             0x3000, 0x4000, 1 << 20, None, 0x10000, 1 << 40, None)
+    assert rc == sparstar.ERR_UNSUPPORTED
+    rc = lib.sparstar_select_ex(0x1000, 0x2000, 1, 256, sparstar.Segments(128, 0, n_kv - 128), 64, 2, 0.05, 0, 96,
+                                0x3000, 0x4000, 1 << 20, None, 0x10000, 1 << 40, None)
+    assert rc == sparstar.ERR_UNSUPPORTED   # block size 96

@@ -247,3 +247,46 @@ def test_schedule_scales(S, scale_index, layer):
               qblocks_per_head=_sampled, heads=[0, 31])
     del q, k, v
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("n_cand", [2048, 2049])
+def test_topk_path_boundary(S, n_cand):
+    """2,048 candidates is the largest row the warp Top-K takes (64 keys per lane); 2,049 goes
+    to the CTA-per-row radix Top-K. Both must give the oracle's masks."""
+    n_text, n_q = 128, 256
+    q, k, v = synth.make_qkv(n_q, n_text + 128 * n_cand, 1, 64, [4000 + n_cand], device="cuda")
+    stats = _run_case(S, q, k, v, n_text, 0, 128 * n_cand, 2, 0.05, 0)
+    assert stats["rows"] == 2
+
+
+@pytest.mark.slow
+def test_max_candidates(S):
+    """16,384 candidates per row (the radix Top-K's shared-memory limit), 2.1 M KV tokens."""
+    n_text, n_cand = 128, 16384
+    q, k, v = synth.make_qkv(200, n_text + 128 * n_cand, 1, 64, [4321], device="cuda")
+    stats = _run_case(S, q, k, v, n_text, 0, 128 * n_cand, 2, 0.01, 0)
+    assert stats["rows"] == 2
+    del q, k, v
+    torch.cuda.empty_cache()
+
+
+def test_wider_index_buffer_and_single_head(S):
+    """kmax larger than K_total: only the first K_total entries of a row are written, the rest
+    keep the caller's values, and attention reads only cnt entries; one head, one query row."""
+    n_text, n_ctx, n_cur = 128, 256, 513
+    q, k, v = synth.make_qkv(1, n_text + n_ctx + n_cur, 1, 128, [77], device="cuda")
+    plan = S.make_plan(1, n_text, n_ctx, n_cur, 2, 0.4)
+    kt = int(plan.k_total)
+    idx = torch.full((1, 1, kt + 5), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    S.select(q, k, n_text, n_ctx, n_cur, 2, 0.4, idx=idx, cnt=cnt)
+    o, lse = S.attn(q, k, v, idx, cnt)
+    assert S.device_status() == S.OK
+    g = idx.cpu().numpy()[0, 0]
+    assert (g[kt:] == -7).all() and int(cnt.item()) == kt
+    qf, kf, vf = (O.bf16_bits_to_f64(bits(x)[0]) for x in (q, k, v))
+    rows, _ = O.select_head(qf, kf, n_text, n_ctx, 2, 0.4)
+    assert np.array_equal(g[:kt], rows[0])
+    (o_ref, lse_ref), = O.block_sparse_attention(qf, kf, vf, rows, [0])
+    check_output(o.float().cpu().numpy()[0], o_ref, "single row")
+    assert abs(float(lse.cpu()[0, 0]) - float(lse_ref[0])) <= LSE_ABS
