@@ -496,13 +496,17 @@ def run_ours(args, rank, world, local_rank):
                     "(model activations) are context only"}
         del dlse, e_block, u_block
 
-    # end to end through the public API with host buffers: H2D of q/k/v, forward, D2H of o
+    # End to end through the public API with host buffers: every step copies its q/k/v from
+    # pinned host memory, runs the forward and reads o back. Heads are independent, so the
+    # step is issued in head chunks on three streams: the H2D copy of chunk c+1 (and of the
+    # next step) overlaps the forward of chunk c and the D2H copy of chunk c-1. The serial
+    # form (copy all, forward, read back) is reported next to it.
     if not args.no_e2e:
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         n_e2e = max(2, min(args.steps, 5))
 
-        def e2e_step():
+        def e2e_serial_step():
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
@@ -510,20 +514,67 @@ def run_ours(args, rank, world, local_rank):
                       o=o, lse=lse)
             ho.copy_(o, non_blocking=True)
 
-        e2e_step()
+        e2e_serial_step()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n_e2e):
-            e2e_step()
+            e2e_serial_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        serial_ms = a.elapsed_time(b) / n_e2e
+
+        n_chunks = min(4, sc.heads)
+        bounds = [(sc.heads * c // n_chunks, sc.heads * (c + 1) // n_chunks) for c in range(n_chunks)]
+        ws_c = S.Workspace(max(h1 - h0 for h0, h1 in bounds), sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
+        s_h2d, s_cmp, s_d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
+        done_cmp = [None] * n_chunks   # forward of chunk c finished (its inputs may be overwritten)
+        done_d2h = [None] * n_chunks   # o of chunk c read back (it may be overwritten)
+
+        def e2e_pipelined_step():
+            for c, (h0, h1) in enumerate(bounds):
+                with torch.cuda.stream(s_h2d):
+                    if done_cmp[c] is not None:
+                        s_h2d.wait_event(done_cmp[c])
+                    q[h0:h1].copy_(hq[h0:h1], non_blocking=True)
+                    k[h0:h1].copy_(hk[h0:h1], non_blocking=True)
+                    v[h0:h1].copy_(hv[h0:h1], non_blocking=True)
+                    ev_in = torch.cuda.Event()
+                    ev_in.record(s_h2d)
+                s_cmp.wait_event(ev_in)
+                if done_d2h[c] is not None:
+                    s_cmp.wait_event(done_d2h[c])
+                S.forward(q[h0:h1], k[h0:h1], v[h0:h1], *seg, sc.clip, sc.density, args.budget_mode, workspace=ws_c,
+                          idx=idx[h0:h1], cnt=cnt[h0:h1], o=o[h0:h1], lse=lse[h0:h1], stream=s_cmp)
+                ev_c = torch.cuda.Event()
+                ev_c.record(s_cmp)
+                done_cmp[c] = ev_c
+                with torch.cuda.stream(s_d2h):
+                    s_d2h.wait_event(ev_c)
+                    ho[h0:h1].copy_(o[h0:h1], non_blocking=True)
+                    ev_o = torch.cuda.Event()
+                    ev_o.record(s_d2h)
+                done_d2h[c] = ev_o
+
+        e2e_pipelined_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_h2d)
+        for _ in range(n_e2e):
+            e2e_pipelined_step()
+        for st in (s_h2d, s_cmp, s_d2h):
+            stream.wait_stream(st)
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems, = max_over_ranks([a.elapsed_time(b) / n_e2e], dev, world)
+        ems, serial_ms = max_over_ranks([a.elapsed_time(b) / n_e2e, serial_ms], dev, world)
         result["e2e"] = {"value": whole_job_tflops(flops, ems, world), "unit": "TFLOP/s",
                          "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
-                         "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e}
-        del hq, hk, hv, ho
+                         "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e,
+                         "pipelined": f"{n_chunks} head chunks per step on three streams (H2D / forward / D2H)",
+                         "serial_value": whole_job_tflops(flops, serial_ms, world), "serial_ms_per_step": serial_ms}
+        del hq, hk, hv, ho, ws_c
 
     if world == 1 and not args.no_schedule and not args.heads:
         del o, lse
