@@ -132,24 +132,22 @@ def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
 
 # --------------------------------------------------------------------------- steps 4-5
 
-def _order_scores(s: np.ndarray) -> np.ndarray:
-    # -0.0 and +0.0 are the same score; NaN (never produced from finite inputs) ranks last.
-    s = np.where(np.isnan(s), -np.inf, s)
-    return s + 0.0
-
-
 def select_rows(S: np.ndarray, n_forced: int, k_topk: int) -> np.ndarray:
     """Kept KV blocks of each query-block row, ascending (方法概览: clip-aware retention + joint Top-K).
 
     S is [nqb, nkb]. The forced blocks 0..n_forced-1 are always kept. The K_topk
     highest-scoring remaining blocks join them; among equal scores the lower block index
-    comes first. The ranking is one library sort per row on the key (-score, index).
+    comes first; -0.0 and +0.0 are the same score; NaN (never produced from finite inputs)
+    ranks below every number, -inf included. The ranking is one library sort per row on the
+    key (is NaN, -score, index).
     """
     nqb, nkb = S.shape
     n_forced = min(n_forced, nkb)
-    cand = _order_scores(S[:, n_forced:])
+    cand = S[:, n_forced:]
+    is_nan = np.isnan(cand)
+    value = np.where(is_nan, 0.0, cand) + 0.0             # + 0.0 turns -0.0 into +0.0
     index = np.broadcast_to(np.arange(n_forced, nkb), cand.shape)
-    order = np.lexsort((index, -cand), axis=-1)          # primary key last: -score, then index
+    order = np.lexsort((index, -value, is_nan), axis=-1)  # primary key last
     chosen = np.sort(order[:, :k_topk] + n_forced, axis=1)
     forced = np.broadcast_to(np.arange(n_forced), (nqb, n_forced))
     return np.concatenate([forced, chosen], axis=1).astype(np.int64)

@@ -158,6 +158,44 @@ def test_topk_signed_zero_ties_and_lower_index():
     assert O.select_row(np.array([5.0, 1.0, np.nan, 0.5]), 0, 3).tolist() == [0, 1, 3]
 
 
+def _beats(a, ia, b, ib):
+    """Pairwise ranking: a number beats NaN; between numbers the larger wins (-0.0 == +0.0);
+    equal scores, and two NaNs, go to the lower index."""
+    na, nb = math.isnan(a), math.isnan(b)
+    if na != nb:
+        return nb
+    if not na and a != b:
+        return a > b
+    return ia < ib
+
+
+def _dominance_choice(scores, n_forced, k_topk):
+    """The unique subset of k_topk candidates each of which beats every unchosen candidate."""
+    cands = list(range(n_forced, len(scores)))
+    found = [sub for sub in itertools.combinations(cands, k_topk)
+             if all(_beats(scores[c], c, scores[u], u) for c in sub for u in cands if u not in sub)]
+    assert len(found) == 1
+    return list(range(n_forced)) + list(found[0])
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_topk_special_values_match_pairwise_dominance(seed):
+    # NaN, +-inf and +-0 mixed with small integers (frequent ties)
+    rng = np.random.default_rng(1000 + seed)
+    nkb = int(rng.integers(2, 11))
+    n_forced = int(rng.integers(0, nkb))
+    k_topk = int(rng.integers(0, nkb - n_forced + 1))
+    pool = np.array([np.nan, np.inf, -np.inf, 0.0, -0.0, 1.0, -1.0, 2.0])
+    scores = rng.choice(pool, size=nkb)
+    got = O.select_row(scores, n_forced, k_topk).tolist()
+    assert got == _dominance_choice(scores.tolist(), n_forced, k_topk)
+
+
+def test_topk_nan_below_negative_infinity():
+    assert O.select_row(np.array([np.nan, -np.inf]), 0, 1).tolist() == [1]
+    assert O.select_row(np.array([np.nan, -np.inf, np.nan]), 0, 2).tolist() == [0, 1]
+
+
 def test_forced_only_rows_ignore_values():
     rng = np.random.default_rng(7)
     for _ in range(10):
