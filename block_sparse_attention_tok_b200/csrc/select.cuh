@@ -16,11 +16,13 @@
 //                    tcgen05.mma accumulating hi.hi + hi.lo + lo.hi in fp32 tensor memory
 //                    (the dropped lo.lo term and the bf16 rounding of lo keep the error near
 //                    2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
-//   topk_warp_kernel one warp per (head, query block) row: the K-th largest key is bracketed
-//                    by a value histogram, then resolved among <= 32 keys by a warp bitonic
-//                    sort; ties taken lowest index first, ascending emit.
+//   topk_warp_kernel one warp per (head, query block) row, staged in shared memory with
+//                    16-byte copies, each lane owning a contiguous run: the K-th largest key
+//                    is bracketed by a value histogram, then resolved among <= 32 keys by a
+//                    warp bitonic sort; ties taken lowest index first; each lane marks its
+//                    taken candidates in a bit mask and one warp scan places the runs.
 //   topk_kernel      one CTA per row, 8-bit radix select in shared memory (rows with more than
-//                    2048 candidates).
+//                    2045 candidates).
 //   fill_kernel      rows that do not depend on scores (K_topk == 0 or every block kept):
 //                    the row is the identity prefix 0..K_total-1.
 #pragma once
@@ -488,78 +490,39 @@ __global__ void __launch_bounds__(128) fill_kernel(int k_total, int32_t* __restr
   if (threadIdx.x == 0) cnt[row] = k_total;
 }
 
-// Top-K of one row by one warp; the row's scores sit in this warp's shared-memory buffer
-// sv[32 * KPL]. The K-th largest key T is located in steps, all exact:
-//   1. the row's score range is split into 256 equal-width bins; binning is monotone in the
-//      score, so every key in a higher bin is larger than every key in a lower one;
-//   2. a per-warp histogram (`hist`, 256 words) and a warp scan give the bin b* holding the
-//      K-th largest key and the number of keys above it;
-//   3. the indices of the keys in bins >= b* (about K of them) are compacted in index order
-//      into `lst` (uint16, one per candidate at most); every later step reads only this list;
-//   4. the keys of b* are gathered (`gather`, 32 words) and sorted by a warp bitonic network;
-//      if b* holds more than 32 keys, its key range is first narrowed by bisection on counts.
-// Every key > T is taken, and of the keys == T the lowest-index ones; the row is emitted
-// ascending after the forced prefix. Keys: NaN ranks below every number; -0.0 equals +0.0.
-template <int KPL>
-__device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, int n_forced, int n_cand, int k_topk,
-                                              int32_t* __restrict__ out, uint32_t* gather, uint32_t* hist,
-                                              float* sv, uint16_t* lst, uint8_t* bins) {
+// Top-K of one row by one warp. The row is staged in shared memory (`sv`, 32*KPL floats,
+// NaN past the row) and lane l owns the contiguous candidates [l*KPL, (l+1)*KPL), read as
+// float4. The K-th largest key T is located in steps, all exact:
+//   1. the row's score range (NaN ignored);
+//   2. the range is split into 256 equal-width bins (binning is monotone in the score, so
+//      every key of a higher bin is larger than every key of a lower one; NaN and the
+//      padding go to bin 0, the padding is then taken out of its count); a per-warp
+//      histogram and a warp scan give the bin b* holding the K-th largest key and the
+//      count of keys above it; each candidate's bin is kept, four to a word;
+//   3. while the set in question (first b*) holds more than 32 keys, it is narrowed by a
+//      histogram over 256 sub-ranges of its ranking keys;
+//   4. the set's <= 32 keys are sorted by a warp bitonic network; T is read off it, with
+//      the number of keys > T and == T;
+//   5. each lane marks its taken candidates in a bit mask (every key > T and, of the keys
+//      == T, the lowest-index ones); one warp scan of the counts places each lane's run,
+//      and the lanes write their candidates in index order.
+// Keys: NaN ranks below every number; -0.0 equals +0.0. `hist` holds 256 words, `gat` 33
+// (32 keys and a counter), `binw` 8*KPL words (the packed bins).
+__device__ __forceinline__ uint32_t rank_key(float x) { return x != x ? 1u : max(score_key(x), 2u); }
+
+// The number whose ranking key is k (k >= 2; the key of zero gives +0.0).
+__device__ __forceinline__ float key_number(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Bin of the need-th largest key (need >= 1) from a 256-bin histogram, scanning from bin 255
+// down; lane l owns bins 255-8l .. 248-8l. Returns the bin, the count of keys above it and
+// the count inside it (warp-uniform).
+__device__ __forceinline__ void find_bin_desc(const uint32_t* hist, uint32_t need, uint32_t& bin, uint32_t& above,
+                                              uint32_t& inside) {
   const int lane = threadIdx.x & 31;
   const uint32_t full = 0xFFFFFFFFu;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  const uint32_t K = static_cast<uint32_t>(k_topk);
-  // Row -> shared memory with asynchronous 4-byte copies (nothing held in registers).
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = lane + 32 * t;
-    if (j < n_cand)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sv + j)), "l"(srow + n_forced + j)
-                   : "memory");
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncwarp();
-  auto key_of = [](float x) -> uint32_t { return x != x ? 1u : max(score_key(x), 2u); };
-  // 1. score range (fminf/fmaxf skip NaN)
-  float lo_s[4] = {INFINITY, INFINITY, INFINITY, INFINITY}, hi_s[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    if (lane + 32 * t < n_cand) {
-      const float x = sv[lane + 32 * t];
-      lo_s[t & 3] = fminf(lo_s[t & 3], x);
-      hi_s[t & 3] = fmaxf(hi_s[t & 3], x);
-    }
-  }
-  float smin = fminf(fminf(lo_s[0], lo_s[1]), fminf(lo_s[2], lo_s[3]));
-  float smax = fmaxf(fmaxf(hi_s[0], hi_s[1]), fmaxf(hi_s[2], hi_s[3]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    smin = fminf(smin, __shfl_xor_sync(full, smin, off));
-    smax = fmaxf(smax, __shfl_xor_sync(full, smax, off));
-  }
-  const float width = smax - smin;
-  const float scale = width > 0.f ? 256.f / width : 0.f;
-  const float offset = -smin * scale;
-  // Bin of a score: f = (x - min) * 256 / width in [0, 256], rounded to nearest by adding
-  // 1.5 * 2^23 (the integer lands in the low mantissa bits), clamped to 255; monotone in x,
-  // NaN -> 0. Computed once per candidate and kept in shared memory.
-  auto bin_of = [&](float x) -> uint32_t {
-    const float f = fmaf(x, scale, offset);
-    return f != f ? 0u : min(255u, __float_as_uint(f + 12582912.0f) & 0x3FFu);
-  };
-  // 2. histogram and the bin of the K-th largest key
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = lane + 32 * t;
-    if (j < n_cand) {
-      const uint32_t b = bin_of(sv[j]);
-      bins[j] = static_cast<uint8_t>(b);
-      atomicAdd(&hist[b], 1u);
-    }
-  }
-  __syncwarp();
-  uint32_t cnt[8], local = 0;  // lane l owns bins 255-8l .. 248-8l (descending)
+  uint32_t cnt[8], local = 0;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     cnt[e] = hist[255 - 8 * lane - e];
@@ -572,133 +535,311 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ srow, in
     if (lane >= off) inc += n;
   }
   uint32_t before = inc - local;
-  const bool owner = before < K && K <= inc;
-  uint32_t bstar_l = 0, above_l = 0, inbin_l = 0;
+  const bool owner = before < need && need <= inc;
+  uint32_t b_l = 0, a_l = 0, i_l = 0;
   if (owner) {
     bool done = false;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (!done && before + cnt[e] >= K) {
-        bstar_l = 255u - 8u * lane - e;
-        above_l = before;
-        inbin_l = cnt[e];
+      if (!done && before + cnt[e] >= need) {
+        b_l = 255u - 8u * lane - e;
+        a_l = before;
+        i_l = cnt[e];
         done = true;
       }
       before += cnt[e];
     }
   }
   const int src = __ffs(__ballot_sync(full, owner)) - 1;
-  const uint32_t bstar = __shfl_sync(full, bstar_l, src);
-  uint32_t c_hi = __shfl_sync(full, above_l, src);          // #(keys in bins above b*)
-  uint32_t c_lo = c_hi + __shfl_sync(full, inbin_l, src);   // #(keys in bins >= b*)
-  // 3. compact the indices with bin >= b*, in index order
-  uint32_t m = 0;
+  bin = __shfl_sync(full, b_l, src);
+  above = __shfl_sync(full, a_l, src);
+  inside = __shfl_sync(full, i_l, src);
+}
+
+__device__ __forceinline__ uint32_t warp_exclusive_scan(uint32_t v, uint32_t& total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t inc = v;
 #pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    const int j = lane + 32 * t;
-    const bool in = j < n_cand && bins[j] >= bstar;
-    const uint32_t ball = __ballot_sync(full, in);
-    if (in) lst[m + __popc(ball & lt_mask)] = static_cast<uint16_t>(j);
-    m += __popc(ball);
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+    if (lane >= off) inc += n;
   }
-  __syncwarp();
-  // 4. key range of b*, narrowed while it holds more than 32 keys
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (uint32_t e = lane; e < m; e += 32) {
-    const uint32_t j = lst[e];
-    if (bins[j] == bstar) {
-      const uint32_t k = key_of(sv[j]);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
-    }
-  }
-  uint64_t lo = __reduce_min_sync(full, kmin);
-  uint64_t hi = static_cast<uint64_t>(__reduce_max_sync(full, kmax)) + 1u;
-  while (c_lo - c_hi > 32u && hi - lo > 1u) {
-    const uint64_t mid = lo + ((hi - lo) >> 1);
-    uint32_t c = 0;
-    for (uint32_t e = lane; e < m; e += 32) c += key_of(sv[lst[e]]) >= static_cast<uint32_t>(mid) ? 1u : 0u;
-    const uint32_t cm = __reduce_add_sync(full, c);
-    if (cm >= K) {
-      lo = mid;
-      c_lo = cm;
+  total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+  return inc - v;
+}
+
+template <int KPL>
+__device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, int n_cand, int n_forced, int k_topk,
+                                              int32_t* __restrict__ out, float* sv, uint32_t* hist, uint32_t* gat,
+                                              uint32_t* binw) {
+  static_assert(KPL % 4 == 0 && KPL <= 64, "keys per lane: a multiple of 4, at most 64");
+  constexpr int Q = KPL / 4;  // float4 groups per lane
+  const int lane = threadIdx.x & 31;
+  const uint32_t full = 0xFFFFFFFFu;
+  const uint32_t K = static_cast<uint32_t>(k_topk);
+  // Stage the row at slot offset dl = (cand mod 16 bytes) / 4, so that whole 16-byte chunks
+  // inside the row move with one copy each; the ragged first and last chunks move element by
+  // element and every slot outside the row holds NaN. Candidate j sits in slot j + dl
+  // (requires dl + n_cand <= 32 * KPL).
+  const int dl = static_cast<int>((reinterpret_cast<uintptr_t>(cand) >> 2) & 3u);
+  const float* base = cand - dl;  // 16-byte aligned
+#pragma unroll
+  for (int u = 0; u < Q; ++u) {
+    const int c = lane + 32 * u;  // chunk: slots 4c .. 4c+3
+    const int j = 4 * c - dl;     // candidate in its first slot
+    if (j >= 0 && j + 3 < n_cand) {
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sv + 4 * c)), "l"(base + 4 * c)
+                   : "memory");
     } else {
-      hi = mid;
-      c_hi = cm;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (j + e >= 0 && j + e < n_cand)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sv + 4 * c + e)),
+                       "l"(base + 4 * c + e)
+                       : "memory");
+        else
+          sv[4 * c + e] = __uint_as_float(0x7FC00000u);
+      }
     }
   }
-  uint32_t base = 0;
-  for (uint32_t e0 = 0; e0 < m; e0 += 32) {
-    const uint32_t e = e0 + lane;
-    const uint32_t k = e < m ? key_of(sv[lst[e]]) : 0u;
-    const bool in = e < m && k >= lo && static_cast<uint64_t>(k) < hi;
-    const uint32_t ball = __ballot_sync(full, in);
-    const uint32_t at = base + __popc(ball & lt_mask);
-    if (in && at < 32u) gather[at] = k;
-    base += __popc(ball);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
+  if (lane == 0) gat[32] = 0u;
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncwarp();
+  const float4* my = reinterpret_cast<const float4*>(sv) + lane * Q;
+  uint32_t* myb = binw + lane * Q;
+  const int j0 = lane * KPL - dl;  // candidate index of this lane's first slot
+  // 1. score range (fminf/fmaxf skip NaN)
+  float lo0 = INFINITY, lo1 = INFINITY, hi0 = -INFINITY, hi1 = -INFINITY;
+#pragma unroll 3
+  for (int g = 0; g < Q; ++g) {
+    const float4 v = my[g];
+    lo0 = fminf(lo0, fminf(v.x, v.y));
+    lo1 = fminf(lo1, fminf(v.z, v.w));
+    hi0 = fmaxf(hi0, fmaxf(v.x, v.y));
+    hi1 = fmaxf(hi1, fmaxf(v.z, v.w));
   }
-  __syncwarp();
-  uint32_t g = lane < static_cast<int>(min(base, 32u)) ? gather[lane] : 0u;
-  __syncwarp();
+  float smin = fminf(lo0, lo1), smax = fmaxf(hi0, hi1);
 #pragma unroll
-  for (int kk = 2; kk <= 32; kk <<= 1) {
+  for (int off = 16; off > 0; off >>= 1) {
+    smin = fminf(smin, __shfl_xor_sync(full, smin, off));
+    smax = fmaxf(smax, __shfl_xor_sync(full, smax, off));
+  }
+  // 2. value bins: f = fma(x, scale, offset) clamped to [0, 255] (NaN -> 0) and rounded to
+  // nearest by adding 1.5 * 2^23 (the integer lands in the low byte); monotone in x.
+  // First try: bins 1..255 over the upper half [mid, max] of the range and bin 0 for every
+  // key below it, NaN and the padding (bin 0 is not counted). If fewer than K keys reach
+  // bin 1, the K-th largest lies below mid: bin the whole range [min, max] into 0..255
+  // instead, the padding taken out of bin 0 afterwards. A range that is empty, constant or
+  // not finite puts every key in bin 0 of the second form and leaves the work to step 3.
+  auto bin_bits = [](float x, float sc, float of) -> uint32_t {
+    const float f = fminf(fmaxf(fmaf(x, sc, of), 0.f), 255.f);
+    return __float_as_uint(__fadd_rn(f, 12582912.0f));  // bin in the low byte
+  };
+  const float mid = 0.5f * smin + 0.5f * smax;
+  float scale = 255.f / (smax - mid);
+  float offset = 1.f - mid * scale;
+  const bool split_ok = smax > mid && mid > smin && fabsf(scale) <= 3.0e38f && fabsf(offset) <= 3.0e38f;
+  uint32_t bstar = 0, c_hi = 0, nb = 0;
+  bool found = false;
+  if (split_ok) {
+    __syncwarp();
+#pragma unroll 3
+    for (int g = 0; g < Q; ++g) {
+      const float4 v = my[g];
+      const uint32_t b0 = bin_bits(v.x, scale, offset), b1 = bin_bits(v.y, scale, offset);
+      const uint32_t b2 = bin_bits(v.z, scale, offset), b3 = bin_bits(v.w, scale, offset);
+      if (b0 & 0xFFu) atomicAdd(&hist[b0 & 0xFFu], 1u);
+      if (b1 & 0xFFu) atomicAdd(&hist[b1 & 0xFFu], 1u);
+      if (b2 & 0xFFu) atomicAdd(&hist[b2 & 0xFFu], 1u);
+      if (b3 & 0xFFu) atomicAdd(&hist[b3 & 0xFFu], 1u);
+      myb[g] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+    }
+    __syncwarp();
+    uint32_t upper = 0;
 #pragma unroll
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      const uint32_t other = __shfl_xor_sync(full, g, jj);
-      const bool descending_block = (lane & kk) == 0;
-      const bool first = (lane & jj) == 0;
-      g = (first == descending_block) ? max(g, other) : min(g, other);
+    for (int e = 0; e < 8; ++e) upper += hist[lane * 8 + e];
+    upper = __reduce_add_sync(full, upper);
+    if (upper >= K) {
+      find_bin_desc(hist, K, bstar, c_hi, nb);
+      found = true;
     }
   }
-  // need-th largest inside the range (1 <= need <= 32 because c_lo >= K > c_hi); a range
-  // narrowed to one key value (possibly held by more than 32 candidates) is T itself.
-  const uint32_t need = K - c_hi;
-  const uint32_t T_sorted = __shfl_sync(full, g, static_cast<int>(min(need, 32u)) - 1);
-  const uint32_t T = (hi - lo == 1u) ? static_cast<uint32_t>(lo) : T_sorted;
-  // 5. emit: every listed key > T and the lowest-index keys == T, in index order
-  uint32_t n_gt = 0;
-  for (uint32_t e = lane; e < m; e += 32) n_gt += key_of(sv[lst[e]]) > T ? 1u : 0u;
-  const uint32_t need_eq = K - __reduce_add_sync(full, n_gt);
+  if (!found) {
+    scale = 256.f / (smax - smin);
+    offset = -smin * scale;
+    if (!(smax > smin) || !(fabsf(scale) <= 3.0e38f) || !(fabsf(offset) <= 3.0e38f)) {
+      scale = 0.f;
+      offset = 0.f;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
+    __syncwarp();
+#pragma unroll 3
+    for (int g = 0; g < Q; ++g) {
+      const float4 v = my[g];
+      const uint32_t b0 = bin_bits(v.x, scale, offset), b1 = bin_bits(v.y, scale, offset);
+      const uint32_t b2 = bin_bits(v.z, scale, offset), b3 = bin_bits(v.w, scale, offset);
+      atomicAdd(&hist[b0 & 0xFFu], 1u);
+      atomicAdd(&hist[b1 & 0xFFu], 1u);
+      atomicAdd(&hist[b2 & 0xFFu], 1u);
+      atomicAdd(&hist[b3 & 0xFFu], 1u);
+      myb[g] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+    }
+    __syncwarp();
+    if (lane == 0) hist[0] -= static_cast<uint32_t>(32 * KPL - n_cand);  // the padding
+    __syncwarp();
+    find_bin_desc(hist, K, bstar, c_hi, nb);
+  }
+  uint32_t need = K - c_hi;  // 1 <= need <= nb
+  auto valid = [&](int j) { return j >= 0 && j < n_cand; };
+  // 3. narrow the set while it holds more than 32 keys: the set's ranking keys span
+  // [klo, khi); each round splits that span into at most 256 sub-ranges of 2^s keys.
+  bool by_key = false;
+  uint32_t klo = 0;
+  uint64_t khi = 0;
+  if (nb > 32u) {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    for (int i = 0; i < KPL; ++i) {
+      if (valid(j0 + i) && ((myb[i >> 2] >> (8 * (i & 3))) & 0xFFu) == bstar) {
+        const uint32_t k = rank_key(sv[lane * KPL + i]);
+        mn = min(mn, k);
+        mx = max(mx, k);
+      }
+    }
+    klo = __reduce_min_sync(full, mn);
+    khi = static_cast<uint64_t>(__reduce_max_sync(full, mx)) + 1u;
+    by_key = true;
+    while (nb > 32u && khi - klo > 1u) {
+      const uint64_t span = khi - klo;
+      const int bits = 64 - __clzll(static_cast<long long>(span - 1u));
+      const int s = bits > 8 ? bits - 8 : 0;
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
+      __syncwarp();
+      for (int i = 0; i < KPL; ++i) {
+        const uint32_t k = rank_key(sv[lane * KPL + i]);
+        if (valid(j0 + i) && k >= klo && static_cast<uint64_t>(k) < khi) atomicAdd(&hist[(k - klo) >> s], 1u);
+      }
+      __syncwarp();
+      uint32_t b2, a2, n2;
+      find_bin_desc(hist, need, b2, a2, n2);
+      const uint64_t kb = klo;
+      klo = static_cast<uint32_t>(kb + (static_cast<uint64_t>(b2) << s));
+      const uint64_t top = kb + (static_cast<uint64_t>(b2 + 1u) << s);
+      khi = top < khi ? top : khi;
+      c_hi += a2;
+      need -= a2;
+      nb = n2;
+    }
+  }
+  // 4. T = the need-th largest key of the set
+  uint32_t T, gt_set, eq_set;
+  if (by_key && khi - klo == 1u) {
+    T = klo;  // every key of the set is equal
+    gt_set = 0;
+    eq_set = nb;
+  } else {
+    if (by_key) {
+      for (int i = 0; i < KPL; ++i) {
+        const uint32_t k = rank_key(sv[lane * KPL + i]);
+        if (valid(j0 + i) && k >= klo && static_cast<uint64_t>(k) < khi) gat[atomicAdd(&gat[32], 1u)] = k;
+      }
+    } else {
+      const uint32_t rep = bstar * 0x01010101u;
+#pragma unroll 3
+      for (int g = 0; g < Q; ++g) {
+        uint32_t m = __vcmpeq4(myb[g], rep);  // 0xFF in each byte whose bin is b*
+        while (m != 0u) {
+          const int e = (__ffs(m) - 1) >> 3;
+          m &= ~(0xFFu << (8 * e));
+          if (valid(j0 + 4 * g + e)) gat[atomicAdd(&gat[32], 1u)] = rank_key(sv[lane * KPL + 4 * g + e]);
+        }
+      }
+    }
+    __syncwarp();
+    uint32_t g = lane < static_cast<int>(nb) ? gat[lane] : 0u;
+#pragma unroll
+    for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        const uint32_t other = __shfl_xor_sync(full, g, jj);
+        const bool descending_block = (lane & kk) == 0;
+        const bool first = (lane & jj) == 0;
+        g = (first == descending_block) ? max(g, other) : min(g, other);
+      }
+    }
+    T = __shfl_sync(full, g, static_cast<int>(need) - 1);
+    gt_set = __popc(__ballot_sync(full, lane < static_cast<int>(nb) && g > T));
+    eq_set = __popc(__ballot_sync(full, lane < static_cast<int>(nb) && g == T));
+  }
+  const uint32_t need_eq = need - gt_set;  // keys == T to take, 1 <= need_eq <= eq_set
+  // 5. mark the taken candidates of this lane, then write them in index order
+  uint64_t take = 0;
+  if (need_eq == eq_set && T >= 2u) {
+    // every key == T is taken and T is a number: take x >= T (NaN and padding compare false)
+    const float tf = key_number(T);
+#pragma unroll 3
+    for (int g = 0; g < Q; ++g) {
+      const float4 v = my[g];
+      const uint64_t m4 = (v.x >= tf ? 1u : 0u) | (v.y >= tf ? 2u : 0u) | (v.z >= tf ? 4u : 0u) | (v.w >= tf ? 8u : 0u);
+      take |= m4 << (4 * g);
+    }
+  } else {
+    uint32_t n_eq = 0;
+    for (int i = 0; i < KPL; ++i) n_eq += (valid(j0 + i) && rank_key(sv[lane * KPL + i]) == T) ? 1u : 0u;
+    uint32_t eq_total;
+    uint32_t eq_rank = warp_exclusive_scan(n_eq, eq_total);
+    for (int i = 0; i < KPL; ++i) {
+      if (!valid(j0 + i)) continue;
+      const uint32_t k = rank_key(sv[lane * KPL + i]);
+      bool t = k > T;
+      if (k == T) {
+        t = eq_rank < need_eq;
+        ++eq_rank;
+      }
+      if (t) take |= 1ull << i;
+    }
+  }
   for (int f = lane; f < n_forced; f += 32) out[f] = f;
-  uint32_t pos = static_cast<uint32_t>(n_forced), eq_seen = 0;
+  uint32_t n_take = __popcll(take), total;
+  uint32_t pos = static_cast<uint32_t>(n_forced) + warp_exclusive_scan(n_take, total);
   const uint32_t row_end = static_cast<uint32_t>(n_forced + k_topk);
-  for (uint32_t e0 = 0; e0 < m; e0 += 32) {
-    const uint32_t e = e0 + lane;
-    const uint32_t j = e < m ? lst[e] : 0u;
-    const uint32_t k = e < m ? key_of(sv[j]) : 0u;
-    const uint32_t eq_ball = __ballot_sync(full, e < m && k == T);
-    const bool take = e < m && (k > T || (k == T && eq_seen + __popc(eq_ball & lt_mask) < need_eq));
-    eq_seen += __popc(eq_ball);
-    const uint32_t take_ball = __ballot_sync(full, take);
-    const uint32_t at = pos + __popc(take_ball & lt_mask);
-    if (take && at < row_end) out[at] = n_forced + static_cast<int>(j);
-    pos += __popc(take_ball);
+  while (take != 0ull) {
+    const int i = __ffsll(static_cast<long long>(take)) - 1;
+    take &= take - 1ull;
+    if (pos < row_end) out[pos] = n_forced + j0 + i;
+    ++pos;
   }
 }
 
-template <int KPL>
-constexpr int topk_warp_smem() {
-  // per warp: scores (fp32), the compacted index list (uint16) and the score bins (uint8)
-  return 8 * 32 * KPL * (4 + 2 + 1);
-}
+// One warp per row, kTopkWarps rows per CTA; grid.x = ceil(H * nqb / kTopkWarps). Requires
+// 1 <= k_topk < n_cand and n_cand + 3 <= 32 * KPL (room for the row's slot offset).
+constexpr int kTopkWarps = 4;
 
-// One warp per row, 8 rows per 256-thread CTA; grid.x = ceil(H * nqb / 8). Requires
-// 1 <= k_topk < n_cand <= 32 * KPL.
 template <int KPL>
-__global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict__ S, int64_t rows, int nkb,
-                                                        int n_forced, int k_topk, int32_t* __restrict__ idx,
-                                                        int32_t* __restrict__ cnt, int kmax) {
-  __shared__ uint32_t gather[8][32];
-  __shared__ uint32_t hist[8][256];
-  extern __shared__ float rowbuf[];  // [8][32 * KPL] scores, then [8][32 * KPL] uint16 lists
+struct TopkSmem {
+  alignas(16) float sv[kTopkWarps][32 * KPL];
+  uint32_t binw[kTopkWarps][8 * KPL];
+  uint32_t hist[kTopkWarps][256];
+  uint32_t gat[kTopkWarps][33];
+};
+
+template <int KPL>
+__global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const float* __restrict__ S, int64_t rows,
+                                                                    int nkb, int n_forced, int k_topk,
+                                                                    int32_t* __restrict__ idx,
+                                                                    int32_t* __restrict__ cnt, int kmax) {
+  __shared__ TopkSmem<KPL> sm;
   const int w = threadIdx.x >> 5;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + w;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kTopkWarps + w;
   griddep_wait();  // scores come from the preceding score kernel
   if (row >= rows) return;
-  uint16_t* lists = reinterpret_cast<uint16_t*>(rowbuf + 8 * 32 * KPL);
-  uint8_t* bins = reinterpret_cast<uint8_t*>(lists + 8 * 32 * KPL);
-  topk_row_warp<KPL>(S + row * nkb, n_forced, nkb - n_forced, k_topk, idx + row * kmax, gather[w], hist[w],
-                     rowbuf + w * 32 * KPL, lists + w * 32 * KPL, bins + w * 32 * KPL);
+  topk_row_warp<KPL>(S + row * nkb + n_forced, nkb - n_forced, n_forced, k_topk, idx + row * kmax, sm.sv[w],
+                     sm.hist[w], sm.gat[w], sm.binw[w]);
   if ((threadIdx.x & 31) == 0) cnt[row] = n_forced + k_topk;
 }
 

@@ -97,10 +97,6 @@ int set_kernel_attrs(DeviceInfo* d) {
                              ScoreConfig<64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMaxCandidates * 4)) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(topk_warp_kernel<36>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             topk_warp_smem<36>()) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(topk_warp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             topk_warp_smem<64>()) == cudaSuccess;
   if (!ok) return SPARSTAR_ERR_CUDA;
   d->attrs_set = true;
   return SPARSTAR_OK;
@@ -160,11 +156,40 @@ cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
 // Keys per lane of the warp Top-K: the smallest supported count that covers n_cand
 // candidates, or 0 when the shared-memory radix kernel has to be used.
 int topk_keys_per_lane(int64_t n_cand) {
-  if (n_cand <= 32 * 8) return 8;
-  if (n_cand <= 32 * 16) return 16;
-  if (n_cand <= 32 * 36) return 36;
-  if (n_cand <= 32 * 64) return 64;
+  for (int kpl : {8, 16, 24, 36, 48, 64})
+    if (n_cand <= 32 * kpl) return kpl;
   return 0;
+}
+
+// Top-K of `rows` score rows of nkb columns (1 <= k_topk < nkb - n_forced <= kMaxCandidates):
+// one warp per row up to 2045 candidates, else one CTA per row. Launched with programmatic
+// stream serialization, so it may start while a preceding score kernel drains.
+void launch_topk(const float* S, int64_t rows, int nkb, int n_forced, int k_topk, int32_t* idx, int32_t* cnt,
+                 int kmax, cudaStream_t st) {
+  const dim3 wgrid(static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps)), wblock(32 * kTopkWarps);
+  switch (topk_keys_per_lane(nkb - n_forced + 3)) {  // + the staging slot offset (<= 3)
+    case 8:
+      launch_after(topk_warp_kernel<8>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    case 16:
+      launch_after(topk_warp_kernel<16>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    case 24:
+      launch_after(topk_warp_kernel<24>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    case 36:
+      launch_after(topk_warp_kernel<36>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    case 48:
+      launch_after(topk_warp_kernel<48>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    case 64:
+      launch_after(topk_warp_kernel<64>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
+      break;
+    default:
+      launch_after(topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(128),
+                   static_cast<size_t>(nkb - n_forced) * 4, st, S, nkb, n_forced, k_topk, idx, cnt, kmax);
+  }
 }
 
 int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, unsigned box_rows = 128) {
@@ -322,28 +347,7 @@ int sparstar_select_ex(const void* q, const void* k, int heads, int64_t n_q, spa
     if ((rc = launch_status()) != SPARSTAR_OK) return rc;
     if (needs_scores) {
       const int n_forced = static_cast<int>(plan.n_forced);
-      const unsigned tgrid = static_cast<unsigned>((rows + 7) / 8);
-      switch (topk_keys_per_lane(plan.n_cand)) {
-        case 8:
-          launch_after(topk_warp_kernel<8>, dim3(tgrid), dim3(256), topk_warp_smem<8>(), st, S, rows, nkb, n_forced,
-                       plan.k_topk, idx, cnt, kmax);
-          break;
-        case 16:
-          launch_after(topk_warp_kernel<16>, dim3(tgrid), dim3(256), topk_warp_smem<16>(), st, S, rows, nkb, n_forced,
-                       plan.k_topk, idx, cnt, kmax);
-          break;
-        case 36:
-          launch_after(topk_warp_kernel<36>, dim3(tgrid), dim3(256), topk_warp_smem<36>(), st, S, rows, nkb, n_forced,
-                       plan.k_topk, idx, cnt, kmax);
-          break;
-        case 64:
-          launch_after(topk_warp_kernel<64>, dim3(tgrid), dim3(256), topk_warp_smem<64>(), st, S, rows, nkb, n_forced,
-                       plan.k_topk, idx, cnt, kmax);
-          break;
-        default:
-          launch_after(topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(128), static_cast<size_t>(plan.n_cand) * 4, st,
-                       S, nkb, n_forced, plan.k_topk, idx, cnt, kmax);
-      }
+      launch_topk(S, rows, nkb, n_forced, static_cast<int>(plan.k_topk), idx, cnt, kmax, st);
       return launch_status();
     }
   }
@@ -356,6 +360,31 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q, sparst
                     float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   return sparstar_select_ex(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, SPARSTAR_BLOCK, idx, cnt,
                             kmax, scores, workspace, workspace_bytes, stream);
+}
+
+int sparstar_topk(const float* scores, int64_t rows, int nkb, int n_forced, int k_topk, int32_t* idx, int32_t* cnt,
+                  int32_t kmax, void* stream) {
+  if (rows < 0 || nkb < 1 || n_forced < 0 || n_forced > nkb || k_topk < 0 || k_topk > nkb - n_forced ||
+      kmax < n_forced + k_topk)
+    return SPARSTAR_ERR_ARG;
+  const int n_cand = nkb - n_forced;
+  const bool reads_scores = k_topk > 0 && k_topk < n_cand;
+  if (rows > INT32_MAX || (reads_scores && n_cand > kMaxCandidates)) return SPARSTAR_ERR_UNSUPPORTED;
+  if (rows == 0) return SPARSTAR_OK;
+  if (idx == nullptr || cnt == nullptr ||
+      (reads_scores && (scores == nullptr || (reinterpret_cast<uintptr_t>(scores) & 3u) != 0)))
+    return SPARSTAR_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;
+  if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (reads_scores)
+    launch_topk(scores, rows, nkb, n_forced, k_topk, idx, cnt, kmax, st);
+  else
+    fill_kernel<<<static_cast<unsigned>(rows), 128, 0, st>>>(n_forced + k_topk, idx, cnt, kmax);
+  return launch_status();
 }
 
 int sparstar_attn_ex(const void* q, const void* k, const void* v, int heads, int64_t n_q, int64_t n_kv, int head_dim,

@@ -83,6 +83,8 @@ _SIGNATURES.update({
     "sparstar_token_bound": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
                                         _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_float, _c.c_void_p,
                                         _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "sparstar_topk": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _c.c_void_p, _c.c_void_p,
+                                 _c.c_int32, _c.c_void_p]),
 })
 NOALLOC_SCRATCH_BYTES = 128 << 20
 
@@ -207,6 +209,26 @@ def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, c
                                    _ptr(cnt), idx.shape[-1], float(sm_scale), _ptr(o), _ptr(lse), _stream_ptr(stream)),
            "sparstar_attn_ex")
     return o, lse
+
+
+def topk(scores: torch.Tensor, n_forced: int, k_topk: int, idx: Optional[torch.Tensor] = None,
+         cnt: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Clip-aware retention + joint Top-K on given scores [..., nkb] (fp32, contiguous CUDA):
+    each row keeps blocks 0..n_forced-1 and its k_topk best other columns, ascending.
+    Returns (idx int32 [..., n_forced + k_topk] unless a wider idx is given, cnt int32 [...])."""
+    if scores.dtype != torch.float32 or not scores.is_cuda or not scores.is_contiguous() or scores.dim() < 1:
+        raise ValueError("scores must be a contiguous fp32 CUDA tensor [..., nkb]")
+    lead, nkb = tuple(scores.shape[:-1]), scores.shape[-1]
+    rows = scores.numel() // nkb if nkb else 0
+    if idx is None:
+        idx = torch.empty(*lead, n_forced + k_topk, dtype=torch.int32, device=scores.device)
+    if cnt is None:
+        cnt = torch.empty(*lead, dtype=torch.int32, device=scores.device)
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous() or not cnt.is_contiguous():
+        raise ValueError("idx/cnt must be contiguous int32")
+    _check(load().sparstar_topk(_ptr(scores), rows, nkb, int(n_forced), int(k_topk), _ptr(idx), _ptr(cnt),
+                                idx.shape[-1], _stream_ptr(stream)), "sparstar_topk")
+    return idx, cnt
 
 
 def _check_lse(*ts):

@@ -113,6 +113,22 @@ int sparstar_select(const void* q, const void* k, int heads, int64_t n_q,
                     int budget_mode, int32_t* idx, int32_t* cnt, int32_t kmax,
                     float* scores, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Clip-aware retention and joint Top-K on scores the caller supplies (digest, 方法概览: the
+ * forced blocks are kept, the rest of each row is filled by a joint Top-K; the selection
+ * steps of sparstar_select without pooling and scoring). scores: fp32 [rows, nkb] device,
+ * 4-byte aligned; columns 0..n_forced-1 are the forced blocks and are not read. Row r of
+ * idx [rows, kmax] receives 0..n_forced-1, then the k_topk highest-scoring columns in
+ * [n_forced, nkb) in ascending order: equal scores go to the lower column, NaN ranks below
+ * every number, -0.0 equals +0.0. cnt[r] = n_forced + k_topk. Entries of idx past that
+ * count are not written. The result is exact: no tolerance applies to the ranking.
+ * Requirements: rows >= 0, 0 <= n_forced <= nkb, 0 <= k_topk <= nkb - n_forced,
+ * kmax >= n_forced + k_topk (else SPARSTAR_ERR_ARG); rows <= 2^31 - 1 and, when the scores
+ * are read (0 < k_topk < nkb - n_forced), nkb - n_forced <= 16384 (else
+ * SPARSTAR_ERR_UNSUPPORTED); scores may be NULL when they are not read. rows == 0 is a
+ * no-op. Requires an sm_100 device. */
+int sparstar_topk(const float* scores, int64_t rows, int nkb, int n_forced, int k_topk,
+                  int32_t* idx, int32_t* cnt, int32_t kmax, void* stream);
+
 /* Forward-only block-sparse attention over the kept tiles (digest, 方法概览 bullet
  * FastFlex执行路径: attention executed over the selected blocks only, with online softmax).
  * For every valid query token t of query block i of head h:

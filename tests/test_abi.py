@@ -141,3 +141,27 @@ def test_select_rejects_more_candidates_than_supported_before_launch(lib):
     rc = lib.sparstar_select_ex(0x1000, 0x2000, 1, 256, sparstar.Segments(128, 0, n_kv - 128), 64, 2, 0.05, 0, 96,
                                 0x3000, 0x4000, 1 << 20, None, 0x10000, 1 << 40, None)
     assert rc == sparstar.ERR_UNSUPPORTED   # block size 96
+
+
+@pytest.mark.parametrize("args,code", [
+    # (rows, nkb, n_forced, k_topk, kmax)
+    ((-1, 10, 2, 3, 8), sparstar.ERR_ARG),          # negative rows
+    ((4, 0, 0, 0, 8), sparstar.ERR_ARG),            # no columns
+    ((4, 10, 11, 0, 16), sparstar.ERR_ARG),         # more forced blocks than columns
+    ((4, 10, -1, 3, 8), sparstar.ERR_ARG),
+    ((4, 10, 2, 9, 16), sparstar.ERR_ARG),          # k_topk > n_cand
+    ((4, 10, 2, -1, 16), sparstar.ERR_ARG),
+    ((4, 10, 2, 3, 4), sparstar.ERR_ARG),           # kmax < n_forced + k_topk
+    ((4, 1 + 16385, 1, 5, 8), sparstar.ERR_UNSUPPORTED),   # 16,385 candidates, scores read
+    ((1 << 31, 10, 2, 3, 8), sparstar.ERR_UNSUPPORTED),    # rows beyond a grid dimension
+])
+def test_topk_rejects_bad_arguments_before_launch(lib, args, code):
+    rows, nkb, n_forced, k_topk, kmax = args
+    assert lib.sparstar_topk(0x1000, rows, nkb, n_forced, k_topk, 0x2000, 0x3000, kmax, None) == code
+
+
+def test_topk_null_and_misaligned_pointers(lib):
+    assert lib.sparstar_topk(None, 4, 10, 2, 3, 0x2000, 0x3000, 8, None) == sparstar.ERR_ARG      # scores read
+    assert lib.sparstar_topk(0x1002, 4, 10, 2, 3, 0x2000, 0x3000, 8, None) == sparstar.ERR_ARG    # not 4-byte aligned
+    assert lib.sparstar_topk(0x1000, 4, 10, 2, 3, None, 0x3000, 8, None) == sparstar.ERR_ARG
+    assert lib.sparstar_topk(0x1000, 0, 10, 2, 3, None, None, 8, None) == sparstar.OK             # rows == 0: no-op
