@@ -146,9 +146,11 @@ struct ScoreConfig {
 // hi.hi + hi.lo + lo.hi bf16 products (fp32 accumulation in tensor memory). Persistent: CTA c
 // takes a contiguous run of tiles in (head, query tile, KV tile) order, so consecutive tiles
 // share the query tile, which stays in shared memory; KV tiles stream through a two-stage
-// TMA ring while the previous tile's epilogue (tensor memory -> registers -> a padded staging
-// buffer -> coalesced rows of S) runs on the other accumulator. Out-of-range rows load as
-// zero and are not stored.
+// TMA ring while the previous tile's epilogue runs on the other accumulator. The epilogue
+// thread of each row takes the row out of tensor memory, frees the accumulator and writes
+// the row with 16-byte stores when rows of S are 16-byte aligned (nkb a multiple of 4);
+// otherwise it goes through a padded staging buffer and coalesced 4-byte row stores.
+// Out-of-range rows load as zero and are not stored.
 template <int D>
 __global__ void __launch_bounds__(ScoreConfig<D>::kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_ql,
@@ -309,6 +311,45 @@ __global__ void __launch_bounds__(ScoreConfig<D>::kThreads, 1)
       const int j0 = nt * 128;
       const int n_cols = min(128, nkb - j0);
       const int i_base = mt * 128 + wq * 32;
+      if ((nkb & 3) == 0) {
+        // Rows of S are 16-byte aligned. Each lane takes its whole row (128 columns) out of
+        // tensor memory and frees the accumulator; then, 32 columns at a time, the warp's
+        // 32 rows pass through the staging buffer (row stride 36 floats: the row-wise 16-byte
+        // writes and the line-wise reads are both free of bank conflicts) and every store
+        // instruction writes four whole 128-byte row lines.
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128u * a + 32u * c, r[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&acc_empty[a]);
+        constexpr int kRow4 = 9;  // float4 per staged row
+        float4* st4 = reinterpret_cast<float4*>(stg);
+        const int sub = lane >> 3, chunk = lane & 7;
+#pragma unroll
+        for (int qc = 0; qc < 4; ++qc) {
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            st4[lane * kRow4 + c4] =
+                make_float4(__uint_as_float(r[qc][4 * c4]) * inv_sqrt_d, __uint_as_float(r[qc][4 * c4 + 1]) * inv_sqrt_d,
+                            __uint_as_float(r[qc][4 * c4 + 2]) * inv_sqrt_d,
+                            __uint_as_float(r[qc][4 * c4 + 3]) * inv_sqrt_d);
+          __syncwarp();
+          const int col = 32 * qc + 4 * chunk;
+          if (col < n_cols) {  // n_cols is a multiple of 4 here
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+              const int rr = 4 * s8 + sub;
+              const int i = i_base + rr;
+              if (i < nqb)
+                *reinterpret_cast<float4*>(S + (static_cast<int64_t>(h) * nqb + i) * nkb + j0 + col) =
+                    st4[rr * kRow4 + chunk];
+            }
+          }
+          __syncwarp();
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         uint32_t r[2][32];
