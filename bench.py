@@ -582,12 +582,13 @@ def run_ours(args, rank, world, local_rank):
         result["schedule"] = run_schedule(S, dev, stream)
 
     if rank == 0 and not args.no_cpu_baseline:
-        qc, kc, vc = (x[:2].cpu() for x in (q, k, v))
-        fl, t, t_pro = oracle_sample(qc, kc, vc, sc, [0, 1], 96, args.budget_mode)
+        n_h = min(4, q.shape[0])
+        qc, kc, vc = (x[:n_h].cpu() for x in (q, k, v))
+        fl, t, t_pro = oracle_sample(qc, kc, vc, sc, list(range(n_h)), 160, args.budget_mode)
         result["cpu_baseline"] = {
             "value": fl / t_pro / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": "heads 0-1 of the same input: bf16 widening + full selection (prorated to the sampled "
-                      "rows) + attention of 96 evenly spaced query blocks per head, fp64 numpy; "
+            "sample": f"heads 0-{n_h - 1} of the same input: bf16 widening + full selection (prorated to the "
+                      "sampled rows) + attention of 160 evenly spaced query blocks per head, fp64 numpy; "
                       f"{t:.1f} s of CPU time"}
     if rank == 0:
         print(json.dumps(result), flush=True)

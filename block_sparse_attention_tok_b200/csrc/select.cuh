@@ -18,9 +18,10 @@
 //                    2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
 //   topk_warp_kernel one warp per (head, query block) row, staged in shared memory with
 //                    16-byte copies, each lane owning a contiguous run: the K-th largest key
-//                    is bracketed by a value histogram, then resolved among <= 32 keys by a
-//                    warp bitonic sort; ties taken lowest index first; each lane marks its
-//                    taken candidates in a bit mask and one warp scan places the runs.
+//                    is bracketed by a value histogram, then resolved among <= 32 keys
+//                    (a rank count or a warp bitonic sort); ties taken lowest index first;
+//                    each lane marks its taken candidates in a bit mask, one warp scan places
+//                    the runs and the row leaves with coalesced stores.
 //   topk_kernel      one CTA per row, 8-bit radix select in shared memory (rows with more than
 //                    2045 candidates).
 //   fill_kernel      rows that do not depend on scores (K_topk == 0 or every block kept):
@@ -542,13 +543,14 @@ __global__ void __launch_bounds__(128) fill_kernel(int k_total, int32_t* __restr
 //      count of keys above it; each candidate's bin is kept, four to a word;
 //   3. while the set in question (first b*) holds more than 32 keys, it is narrowed by a
 //      histogram over 256 sub-ranges of its ranking keys;
-//   4. the set's <= 32 keys are sorted by a warp bitonic network; T is read off it, with
-//      the number of keys > T and == T;
+//   4. the set's <= 32 keys are gathered (per-lane counts, one warp scan) and ranked (a
+//      count over the set when it holds at most 12 keys, else a warp bitonic sort); T is
+//      read off it, with the number of keys > T and == T;
 //   5. each lane marks its taken candidates in a bit mask (every key > T and, of the keys
-//      == T, the lowest-index ones); one warp scan of the counts places each lane's run,
-//      and the lanes write their candidates in index order.
-// Keys: NaN ranks below every number; -0.0 equals +0.0. `hist` holds 256 words, `gat` 33
-// (32 keys and a counter), `binw` 8*KPL words (the packed bins).
+//      == T, the lowest-index ones); one warp scan of the counts places each lane's run in
+//      the staging buffer, in index order, and the row leaves with coalesced stores.
+// Keys: NaN ranks below every number; -0.0 equals +0.0. `hist` holds 256 words, `gat` 32
+// (the set's keys), `binw` 8*KPL words (the packed bins).
 __device__ __forceinline__ uint32_t rank_key(float x) { return x != x ? 1u : max(score_key(x), 2u); }
 
 // The number whose ranking key is k (k >= 2; the key of zero gives +0.0).
@@ -645,7 +647,6 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
-  if (lane == 0) gat[32] = 0u;
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncwarp();
   const float4* my = reinterpret_cast<const float4*>(sv) + lane * Q;
@@ -777,45 +778,77 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
       nb = n2;
     }
   }
-  // 4. T = the need-th largest key of the set
+  // 4. T = the need-th largest key of the set: its <= 32 keys are gathered (each lane counts
+  // its members, a warp scan places them), then ranked (a count over the set when it is small,
+  // else a warp bitonic sort).
   uint32_t T, gt_set, eq_set;
   if (by_key && khi - klo == 1u) {
     T = klo;  // every key of the set is equal
     gt_set = 0;
     eq_set = nb;
   } else {
-    if (by_key) {
-      for (int i = 0; i < KPL; ++i) {
+    auto member = [&](int i) -> bool {
+      if (!valid(j0 + i)) return false;
+      if (by_key) {
         const uint32_t k = rank_key(sv[lane * KPL + i]);
-        if (valid(j0 + i) && k >= klo && static_cast<uint64_t>(k) < khi) gat[atomicAdd(&gat[32], 1u)] = k;
+        return k >= klo && static_cast<uint64_t>(k) < khi;
       }
+      return ((myb[i >> 2] >> (8 * (i & 3))) & 0xFFu) == bstar;
+    };
+    const uint32_t rep = bstar * 0x01010101u;
+    // bins can be matched four at a time unless the padding (bin 0 of the whole-range
+    // binning) could be among the matches
+    const bool by_word = !by_key && bstar != 0u;
+    uint32_t n_mine = 0;
+    if (by_word) {
+#pragma unroll 3
+      for (int g = 0; g < Q; ++g) n_mine += __popc(__vcmpeq4(myb[g], rep)) >> 3;
     } else {
-      const uint32_t rep = bstar * 0x01010101u;
+      for (int i = 0; i < KPL; ++i) n_mine += member(i) ? 1u : 0u;
+    }
+    uint32_t n_all;
+    uint32_t at = warp_exclusive_scan(n_mine, n_all);
+    if (by_word) {
 #pragma unroll 3
       for (int g = 0; g < Q; ++g) {
         uint32_t m = __vcmpeq4(myb[g], rep);  // 0xFF in each byte whose bin is b*
         while (m != 0u) {
           const int e = (__ffs(m) - 1) >> 3;
           m &= ~(0xFFu << (8 * e));
-          if (valid(j0 + 4 * g + e)) gat[atomicAdd(&gat[32], 1u)] = rank_key(sv[lane * KPL + 4 * g + e]);
+          gat[at++] = rank_key(sv[lane * KPL + 4 * g + e]);
         }
       }
+    } else if (n_mine != 0u) {
+      for (int i = 0; i < KPL; ++i)
+        if (member(i)) gat[at++] = rank_key(sv[lane * KPL + i]);
     }
     __syncwarp();
-    uint32_t g = lane < static_cast<int>(nb) ? gat[lane] : 0u;
-#pragma unroll
-    for (int kk = 2; kk <= 32; kk <<= 1) {
-#pragma unroll
-      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-        const uint32_t other = __shfl_xor_sync(full, g, jj);
-        const bool descending_block = (lane & kk) == 0;
-        const bool first = (lane & jj) == 0;
-        g = (first == descending_block) ? max(g, other) : min(g, other);
+    const bool in_set = lane < static_cast<int>(nb);
+    uint32_t g = in_set ? gat[lane] : 0u;
+    if (nb <= 12u) {
+      // rank = keys above this one, equal keys at lower lanes counted as above
+      uint32_t rank = 0;
+      for (int m = 0; m < static_cast<int>(nb); ++m) {
+        const uint32_t o = __shfl_sync(full, g, m);
+        rank += (o > g || (o == g && m < lane)) ? 1u : 0u;
       }
+      const uint32_t hit = __ballot_sync(full, in_set && rank == need - 1u);
+      T = __shfl_sync(full, g, __ffs(hit) - 1);
+    } else {
+#pragma unroll
+      for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+          const uint32_t other = __shfl_xor_sync(full, g, jj);
+          const bool descending_block = (lane & kk) == 0;
+          const bool first = (lane & jj) == 0;
+          g = (first == descending_block) ? max(g, other) : min(g, other);
+        }
+      }
+      T = __shfl_sync(full, g, static_cast<int>(need) - 1);
     }
-    T = __shfl_sync(full, g, static_cast<int>(need) - 1);
-    gt_set = __popc(__ballot_sync(full, lane < static_cast<int>(nb) && g > T));
-    eq_set = __popc(__ballot_sync(full, lane < static_cast<int>(nb) && g == T));
+    gt_set = __popc(__ballot_sync(full, in_set && g > T));
+    eq_set = __popc(__ballot_sync(full, in_set && g == T));
   }
   const uint32_t need_eq = need - gt_set;  // keys == T to take, 1 <= need_eq <= eq_set
   // 5. mark the taken candidates of this lane, then write them in index order
@@ -845,16 +878,21 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
       if (t) take |= 1ull << i;
     }
   }
+  // each lane's taken candidates go to its run in the (now free) staging buffer, then the
+  // row leaves with coalesced stores
   for (int f = lane; f < n_forced; f += 32) out[f] = f;
   uint32_t n_take = __popcll(take), total;
-  uint32_t pos = static_cast<uint32_t>(n_forced) + warp_exclusive_scan(n_take, total);
-  const uint32_t row_end = static_cast<uint32_t>(n_forced + k_topk);
+  uint32_t pos = warp_exclusive_scan(n_take, total);
+  int32_t* ordered = reinterpret_cast<int32_t*>(sv);
+  __syncwarp();
   while (take != 0ull) {
     const int i = __ffsll(static_cast<long long>(take)) - 1;
     take &= take - 1ull;
-    if (pos < row_end) out[pos] = n_forced + j0 + i;
+    if (pos < K) ordered[pos] = n_forced + j0 + i;
     ++pos;
   }
+  __syncwarp();
+  for (uint32_t p = lane; p < K; p += 32) out[n_forced + p] = ordered[p];
 }
 
 // One warp per row, kTopkWarps rows per CTA; grid.x = ceil(H * nqb / kTopkWarps). Requires
@@ -866,7 +904,7 @@ struct TopkSmem {
   alignas(16) float sv[kTopkWarps][32 * KPL];
   uint32_t binw[kTopkWarps][8 * KPL];
   uint32_t hist[kTopkWarps][256];
-  uint32_t gat[kTopkWarps][33];
+  uint32_t gat[kTopkWarps][32];
 };
 
 template <int KPL>
