@@ -321,25 +321,37 @@ __global__ void __launch_bounds__(BoundConfig<D>::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&s_free[b]);  // S is in registers: the buffer may be overwritten
-        // Per value one warp-uniform test; the histogram update is predicated, not branched
-        // per lane. tb = grid coordinate inside the interval: (x + 64) * 2^(5p-1) is exact,
-        // and subtracting the integer lo_idx is exact wherever the result can be in [0, 32).
+        // tb = grid coordinate inside the interval: (x + 64) * 2^(5p-1) is exact, and
+        // subtracting the integer lo_idx is exact wherever the result can be in [0, 32).
         // Values above the interval (tb >= 32) were counted by an earlier pass; in pass 0 they
-        // are values above 2^0 by a rounding and go to the top bin.
+        // are values above 2^0 by a rounding and go to the top bin. The in-interval test of
+        // all 64 values comes first (no votes); then one warp-uniform test per group of 8
+        // values skips the groups no lane needs (most of them after pass 0), and inside a
+        // group the histogram update is predicated, not branched per lane.
+        uint32_t in_mask[2] = {0u, 0u};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float x = fmaf(__uint_as_float(r[c][e]), p.scale_log2, x_off);  // log2 P
             const float tb = (x - kBoundLo) * inv_w - lo_f;
-            const bool in = (32 * c + e < cols) && tb >= 0.f && tb < hi_f;
-            if (__any_sync(0xFFFFFFFFu, in)) {
+            if ((32 * c + e < cols) && tb >= 0.f && tb < hi_f) in_mask[c] |= 1u << e;
+          }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (!__any_sync(0xFFFFFFFFu, ((in_mask[c] >> (8 * g)) & 0xFFu) != 0u)) continue;
+#pragma unroll
+            for (int e = 8 * g; e < 8 * g + 8; ++e) {
+              const bool in = (in_mask[c] >> e) & 1u;
+              const float x = fmaf(__uint_as_float(r[c][e]), p.scale_log2, x_off);
+              const float tb = (x - kBoundLo) * inv_w - lo_f;
               const int bin = in ? min(static_cast<int>(tb), kBoundBins - 1) : 0;
               hn[bin * 32] += in ? 1u : 0u;
               hm[bin * 32] += in ? ex2_approx(x) : 0.f;
             }
           }
-        }
       }
       // Both halves of every row are binned: combine and move the interval. The two warps of
       // a lane quarter reach both named barriers on every path (an aborted wait only ends
