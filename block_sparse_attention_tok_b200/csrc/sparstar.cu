@@ -21,6 +21,21 @@ namespace sparstar {
 // library, so no allocation is needed.
 __device__ unsigned g_status = 0u;
 
+// Self-test of the bounded wait: one thread waits, with the library's mbar_wait, on an
+// mbarrier that nothing ever completes. The wait ends at its time limit, raises the CTA's
+// abort flag and records a timeout in the status word; the kernel then returns normally.
+__global__ void wait_timeout_selftest_kernel(unsigned* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0u, &abort_flag, status);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -579,6 +594,15 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
   }
   return sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
                          scratch, SPARSTAR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int sparstar_selftest_wait_timeout(void* stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if (dev->major != 10) return SPARSTAR_ERR_UNSUPPORTED;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->status);
+  return launch_status();
 }
 
 int sparstar_device_status(void* stream, int clear) {

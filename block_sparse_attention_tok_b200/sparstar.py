@@ -58,6 +58,7 @@ _SIGNATURES.update({
                                     _c.c_int, _c.c_double, _c.c_int, _c.c_float, _c.c_void_p, _c.c_void_p,
                                     _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "sparstar_device_status": (_c.c_int, [_c.c_void_p, _c.c_int]),
+    "sparstar_selftest_wait_timeout": (_c.c_int, [_c.c_void_p]),
     "sparstar_make_plan_ex": (_c.c_int, [_c.c_int64, Segments, _c.c_int, _c.c_double, _c.c_int, _c.c_int,
                                          _c.POINTER(Plan)]),
     "sparstar_workspace_size_ex": (_c.c_int, [_c.c_int, _c.c_int64, Segments, _c.c_int, _c.c_int,
@@ -319,6 +320,11 @@ def select_noalloc(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_
 def device_status(clear: bool = True, stream=None) -> int:
     """Synchronize and return the device status code (OK, ERR_DEVICE_TIMEOUT or ERR_DEVICE_BOUNDS)."""
     return int(load().sparstar_device_status(_stream_ptr(stream), 1 if clear else 0))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test: the next device_status() reports ERR_DEVICE_TIMEOUT."""
+    _check(load().sparstar_selftest_wait_timeout(_stream_ptr(stream)), "sparstar_selftest_wait_timeout")
 
 
 def exported_symbols():

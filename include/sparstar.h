@@ -234,6 +234,13 @@ int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, i
  * SPARSTAR_ERR_CUDA if the synchronization itself failed. clear != 0 resets the word. */
 int sparstar_device_status(void* stream, int clear);
 
+/* Self-test of failure reporting: enqueues one thread that waits, with the same bounded
+ * mbarrier wait the kernels use, on a barrier nothing completes. After the wait limit (2 s
+ * of %globaltimer) the thread records a timeout in the device status word and the kernel
+ * returns normally, so a later sparstar_device_status() returns SPARSTAR_ERR_DEVICE_TIMEOUT
+ * and the CUDA context stays usable. Requires an sm_100 device. */
+int sparstar_selftest_wait_timeout(void* stream);
+
 /* Static text for a return code (never NULL). */
 const char* sparstar_strerror(int code);
 

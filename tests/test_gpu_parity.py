@@ -203,6 +203,23 @@ def test_out_of_range_index_is_clamped_and_reported(S):
     assert S.device_status(clear=True) == S.OK
 
 
+def test_bounded_wait_reports_timeout_and_context_survives(S):
+    """A wait on an mbarrier that nothing completes ends at its 2 s limit with a timeout in the
+    status word (no trap, no hang); afterwards the same context still computes correctly."""
+    import time
+    S.device_status(clear=True)
+    t0 = time.perf_counter()
+    S.selftest_wait_timeout()
+    code = S.device_status(clear=True)
+    elapsed = time.perf_counter() - t0
+    assert code == S.ERR_DEVICE_TIMEOUT
+    assert 1.5 < elapsed < 60.0
+    assert S.device_status(clear=True) == S.OK      # the word was cleared
+    q, k, v = synth.make_qkv(640, 1100, 2, 128, [61, 62], device="cuda")
+    stats = _run_case(S, q, k, v, 100, 300, 700, 2, 0.5, 0)
+    assert stats["rows"] == 2 * 5
+
+
 def test_custom_softmax_scale(S):
     q, k, v = synth.make_qkv(300, 700, 1, 128, [51], device="cuda")
     rows = np.array([[[0, 2, 5], [1, 3, 4], [0, 1, 2]]])
