@@ -310,11 +310,52 @@ def mass_report(q: np.ndarray, k: np.ndarray, rows: np.ndarray, qblocks: Sequenc
     return np.array(E), np.array(U), np.concatenate(R_rows), np.concatenate(U_rows)
 
 
+
+def reference_mass(q: np.ndarray, k: np.ndarray, kept_ref_blocks: np.ndarray, n_text: int, n_ctx: int,
+                   qblocks: Sequence[int], sm_scale: float | None = None, block: int = BLOCK) -> np.ndarray:
+    """Retained attention mass over the reference context (关键结果与论文证据, bullet 跨clip边界,
+    Figure 4): for each listed query block i, the mean over its valid rows t of
+    sum_{u in kept reference tokens} P_tu / sum_{u in all reference tokens} P_tu, with P the
+    dense softmax of row t over every KV token and kept_ref_blocks[i] the kept reference
+    blocks (block ids of the whole KV, all inside [n_text, n_text + n_ctx))."""
+    ref = np.arange(n_text, n_text + n_ctx)
+    out = []
+    for i in qblocks:
+        s, e = block_token_range(int(i), q.shape[0], block)
+        p = dense_probabilities(q[s:e], k, sm_scale)
+        tokens = kept_token_index(kept_ref_blocks[i], k.shape[0], block)
+        out.append((p[:, tokens].sum(axis=1) / p[:, ref].sum(axis=1)).mean())
+    return np.array(out)
+
+
+def reference_reuse_report(q_now: np.ndarray, q_prev: np.ndarray, k: np.ndarray, n_text: int, n_ctx: int,
+                           budget_frac: float, qblocks: Sequence[int], sm_scale: float | None = None,
+                           block: int = BLOCK):
+    """Fresh against reused selection over the reference context under one reference budget
+    (关键结果与论文证据, bullet 跨clip边界; Figure 4). The reference context of the current clip
+    is the preceding clip's final scale, so its key blocks are the tokens that clip's final
+    scale selected among. Per query block i the budget is ceil(budget_frac * n_ref) of the
+    n_ref reference blocks; fresh: the best of them by the current queries' block scores;
+    reused: the best by the preceding clip's queries of the same query block (same position
+    in the clip). Ties go to the lower index. Segments must be whole blocks.
+    Returns (fresh rows [nqb, K], reused rows [nqb, K], E_fresh, E_reused) with block ids of
+    the whole KV and E over qblocks (reference_mass)."""
+    assert n_text % block == 0 and n_ctx % block == 0 and q_now.shape == q_prev.shape
+    nb_text, n_ref = n_text // block, n_ctx // block
+    k_ref = ceil_exact(budget_frac * n_ref)
+    kbar = pool_blocks(k[n_text:n_text + n_ctx], block)
+    fresh = select_rows(block_scores(pool_blocks(q_now, block), kbar), 0, k_ref) + nb_text
+    reused = select_rows(block_scores(pool_blocks(q_prev, block), kbar), 0, k_ref) + nb_text
+    e_fresh = reference_mass(q_now, k, fresh, n_text, n_ctx, qblocks, sm_scale, block)
+    e_reused = reference_mass(q_now, k, reused, n_text, n_ctx, qblocks, sm_scale, block)
+    return fresh, reused, e_fresh, e_reused
+
 __all__ = [
     "BLOCK", "BUDGET_LITERAL", "BUDGET_CANDIDATES", "bf16_bits_to_f64", "num_blocks",
     "block_token_range", "forced_block_count", "row_budget", "pool_blocks", "block_scores",
     "select_rows", "select_row", "select_head", "select", "kept_token_index", "attend_rows",
     "block_sparse_attention", "dense_attention", "retained_mass", "block_energy",
-    "kept_token_count", "dense_probabilities", "token_topk_bound", "mass_report",
+    "kept_token_count", "dense_probabilities", "token_topk_bound", "mass_report", "reference_mass",
+    "reference_reuse_report",
 ]
 

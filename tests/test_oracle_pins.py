@@ -420,3 +420,47 @@ def test_block_size_consistency_64_vs_128():
     p64, p128 = O.pool_blocks(k, 64), O.pool_blocks(k, 128)
     np.testing.assert_allclose((p64[0::2] + p64[1::2]) / 2, p128, rtol=0, atol=1e-15)
     assert O.forced_block_count(512, 8192, 1, 64) == 2 * O.forced_block_count(512, 8192, 1, 128) == 136
+
+
+# ------------------------------------------------------------------ reference-context reuse
+
+def _reuse_case(seed, n_text=128, n_ctx=512, n_cur=256, nq=384, d=16):
+    rng = np.random.default_rng(seed)
+    k = rng.normal(size=(n_text + n_ctx + n_cur, d))
+    k += np.repeat(rng.normal(scale=0.5, size=(O.num_blocks(k.shape[0]), d)), 128, axis=0)[:k.shape[0]]
+    return rng.normal(size=(nq, d)), rng.normal(size=(nq, d)), k
+
+
+def test_reference_mass_matches_torch_softmax_ratio():
+    q, _, k = _reuse_case(1)
+    n_text, n_ctx = 128, 512
+    kept = np.array([[1, 3], [2, 4], [1, 4]])
+    got = O.reference_mass(q, k, kept, n_text, n_ctx, [0, 1, 2])
+    logits = torch.from_numpy(q @ k.T / math.sqrt(q.shape[1]))
+    p = torch.softmax(logits, dim=1).numpy()
+    for i in range(3):
+        rows = slice(128 * i, 128 * (i + 1))
+        cols = np.concatenate([np.arange(128 * j, 128 * (j + 1)) for j in kept[i]])
+        want = (p[rows][:, cols].sum(axis=1) / p[rows, n_text:n_text + n_ctx].sum(axis=1)).mean()
+        assert got[i] == pytest.approx(want, rel=1e-12)
+
+
+def test_reference_reuse_full_budget_and_identical_queries():
+    q_now, q_prev, k = _reuse_case(2)
+    fresh, reused, ef, er = O.reference_reuse_report(q_now, q_prev, k, 128, 512, 1.0, [0, 1, 2])
+    assert np.allclose(ef, 1.0, atol=1e-14) and np.allclose(er, 1.0, atol=1e-14)   # every block kept
+    fresh, reused, ef, er = O.reference_reuse_report(q_now, q_now, k, 128, 512, 0.5, [0, 1, 2])
+    assert np.array_equal(fresh, reused) and np.array_equal(ef, er)
+
+
+def test_reference_reuse_rows_follow_global_block_scores_and_grow_with_budget():
+    q_now, q_prev, k = _reuse_case(3)
+    fresh, reused, ef, er = O.reference_reuse_report(q_now, q_prev, k, 128, 512, 0.5, [0, 1, 2])
+    # the reference blocks are global blocks 1..4 (text is one block): pooling the segment
+    # alone must agree with the scores of the whole KV
+    S = O.block_scores(O.pool_blocks(q_now), O.pool_blocks(k))[:, 1:5]
+    want = np.sort(np.argsort(-S, axis=1, kind="stable")[:, :2], axis=1) + 1
+    assert np.array_equal(fresh, want)
+    assert fresh.min() >= 1 and fresh.max() <= 4 and reused.min() >= 1 and reused.max() <= 4
+    _, _, ef_small, _ = O.reference_reuse_report(q_now, q_prev, k, 128, 512, 0.25, [0, 1, 2])
+    assert np.all(ef >= ef_small)   # nested Top-K sets keep at least as much mass
