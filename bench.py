@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-block64", action="store_true", help="skip the 64-token block variant")
+    ap.add_argument("--no-reuse", action="store_true",
+                    help="skip the fresh vs reused reference-selection comparison")
     ap.add_argument("--no-schedule", action="store_true",
                     help="skip the per-scale timing of the refined-scale schedule (4 scales x 36 layers)")
     return ap.parse_args()
@@ -495,6 +497,29 @@ def run_ours(args, rank, world, local_rank):
             "note": "per query block means over valid rows; synthetic inputs, so the pages' values "
                     "(model activations) are context only"}
         del dlse, e_block, u_block
+
+    # Fresh against reused selection over the reference context (the digest's cross-clip
+    # comparison, Figure 4): the preceding clip's queries (seeded, independent of the current
+    # clip's: the synthetic inputs carry no correlation between clips) pick the reused pattern.
+    if not args.no_reuse and not args.heads and sc.clip >= 2 and sc.n_text % 128 == 0 and sc.n_ctx % 128 == 0:
+        from block_sparse_attention_tok_b200 import reuse
+        q_prev = synth.make_prev_clip_queries(sc.n_q, sc.heads, sc.head_dim,
+                                              [500000 + h + 1000 * rank for h in range(sc.heads)], device=dev)
+        reuse.reference_reuse(q, q_prev, k, v, *seg, 0.15, workspace=ws)   # warm-up
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        res = reuse.reference_reuse(q, q_prev, k, v, *seg, 0.15, workspace=ws)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        result["reuse"] = {
+            "reference_budget": 0.15, "k_ref": res["k_ref"], "n_ref_blocks": sc.n_ctx // 128,
+            "fresh_mean": float(res["e_fresh"].mean()), "reused_mean": float(res["e_reused"].mean()),
+            "ms": r0.elapsed_time(r1),
+            "note": "retained share of the softmax mass over the reference context; the preceding clip's "
+                    "queries are synthetic and independent of the current ones, so the reused pattern acts "
+                    "as an uninformed one here (the pages' 85% vs 56% come from model activations)"}
+        del q_prev, res
+        torch.cuda.empty_cache()
 
     # End to end through the public API with host buffers: every step copies its q/k/v from
     # pinned host memory, runs the forward and reads o back. Heads are independent, so the

@@ -122,6 +122,19 @@ def make_scale_inputs(scale: Scale, device="cpu", layer: int = 0, scale_index: i
     return make_qkv(scale.n_q, scale.n_kv, H, scale.head_dim, seeds, device)
 
 
+def make_prev_clip_queries(n_q: int, heads: int, d: int, seeds: List[int], device="cpu") -> torch.Tensor:
+    """Queries of the preceding clip's final scale (same shape as the current queries), for the
+    reference-reuse comparison: bf16 [H, Nq, d], N(0,1) per element, one generator per head
+    seeded seeds[h]. Drawn independently of the current clip's inputs (the synthetic inputs
+    carry no correlation between clips)."""
+    q = torch.empty(heads, n_q, d, dtype=torch.bfloat16, device=device)
+    gen = torch.Generator(device=device)
+    for h in range(heads):
+        gen.manual_seed(int(seeds[h]))
+        q[h].copy_(torch.randn(n_q, d, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16))
+    return q
+
+
 def random_small_cases(seed: int = 1234, count: int = 12) -> Iterator[dict]:
     """Small ragged shapes for parity sweeps: H in {1,2}, d in {64,128}, ragged Q/KV tails."""
     g = torch.Generator().manual_seed(seed)
