@@ -9,7 +9,7 @@
 //     sequence of (head, query block) items, so the softmax of one slot overlaps the tensor
 //     core work of the other;
 //   * warp 8 (TMA): loads the slot's 128xd Q tile once per item and, per kept block, the K
-//     and V tiles into a ring of shared-memory stages (128-byte swizzle, no multicast);
+//     and V tiles into a ring of shared-memory stages (128-byte swizzle; each CTA loads its own);
 //   * warp 9 (MMA, one thread): S = Q K^T into tensor memory (tcgen05.mma, M=128, N=128,
 //     K=16 steps), then O += P V with P read from tensor memory;
 //   * warps 0-3 / 4-7 (softmax of slot 0 / 1, one thread per query row): tcgen05.ld of the

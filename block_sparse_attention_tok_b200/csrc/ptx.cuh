@@ -87,7 +87,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled load (no multicast) of one box into shared memory; completes `bar`'s tx count.
+// 3-D tiled load of one box into this CTA's own shared memory; completes `bar`'s tx count.
 // c0 is the innermost (element) coordinate and must be a multiple of 8 for bf16.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2) {
