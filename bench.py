@@ -409,6 +409,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic", "config": workload_config(sc, args),
         "gpu_launches": launches_per_step * args.steps,
         "attn": {"ms": t_att, "tflops": attn_tflops, "frac_of_peak": attn_tflops / peak_t,
+                 "frac_of_burst_peak": attn_tflops / float(peaks["bf16_tflops"]),
                  "kept_tile_tflop": flops / 1e12, "kept_blocks_per_row": kmax},
         "select": {"us": t_sel * 1e3, "gbs": sel_gbs, "frac_of_hbm": sel_gbs / peak_hbm,
                    "bytes": sel_bytes, "share_of_step": t_sel / (t_sel + t_att)},
