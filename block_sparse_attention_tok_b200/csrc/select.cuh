@@ -23,7 +23,7 @@
 //                    each lane marks its taken candidates in a bit mask, one warp scan places
 //                    the runs and the row leaves with coalesced stores.
 //   topk_kernel      one CTA per row, 8-bit radix select in shared memory (rows with more than
-//                    2045 candidates).
+//                    3965 candidates).
 //   fill_kernel      rows that do not depend on scores (K_topk == 0 or every block kept):
 //                    the row is the identity prefix 0..K_total-1.
 #pragma once
@@ -615,7 +615,7 @@ template <int KPL>
 __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, int n_cand, int n_forced, int k_topk,
                                               int32_t* __restrict__ out, float* sv, uint32_t* hist, uint32_t* gat,
                                               uint32_t* binw) {
-  static_assert(KPL % 4 == 0 && KPL <= 64, "keys per lane: a multiple of 4, at most 64");
+  static_assert(KPL % 4 == 0 && KPL <= 128, "keys per lane: a multiple of 4, at most 128 (two take words)");
   constexpr int Q = KPL / 4;  // float4 groups per lane
   const int lane = threadIdx.x & 31;
   const uint32_t full = 0xFFFFFFFFu;
@@ -852,7 +852,7 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
   }
   const uint32_t need_eq = need - gt_set;  // keys == T to take, 1 <= need_eq <= eq_set
   // 5. mark the taken candidates of this lane, then write them in index order
-  uint64_t take = 0;
+  uint64_t take0 = 0, take1 = 0;  // bit i of take0 / take1: candidate j0 + i / j0 + 64 + i taken
   if (need_eq == eq_set && T >= 2u) {
     // every key == T is taken and T is a number: take x >= T (NaN and padding compare false)
     const float tf = key_number(T);
@@ -860,7 +860,10 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
     for (int g = 0; g < Q; ++g) {
       const float4 v = my[g];
       const uint64_t m4 = (v.x >= tf ? 1u : 0u) | (v.y >= tf ? 2u : 0u) | (v.z >= tf ? 4u : 0u) | (v.w >= tf ? 8u : 0u);
-      take |= m4 << (4 * g);
+      if (4 * g < 64)
+        take0 |= m4 << (4 * g);
+      else
+        take1 |= m4 << (4 * g - 64);
     }
   } else {
     uint32_t n_eq = 0;
@@ -875,46 +878,57 @@ __device__ __forceinline__ void topk_row_warp(const float* __restrict__ cand, in
         t = eq_rank < need_eq;
         ++eq_rank;
       }
-      if (t) take |= 1ull << i;
+      if (t) {
+        if (i < 64)
+          take0 |= 1ull << i;
+        else
+          take1 |= 1ull << (i - 64);
+      }
     }
   }
   // each lane's taken candidates go to its run in the (now free) staging buffer, then the
   // row leaves with coalesced stores
   for (int f = lane; f < n_forced; f += 32) out[f] = f;
-  uint32_t n_take = __popcll(take), total;
+  uint32_t n_take = __popcll(take0) + __popcll(take1), total;
   uint32_t pos = warp_exclusive_scan(n_take, total);
   int32_t* ordered = reinterpret_cast<int32_t*>(sv);
   __syncwarp();
-  while (take != 0ull) {
-    const int i = __ffsll(static_cast<long long>(take)) - 1;
-    take &= take - 1ull;
-    if (pos < K) ordered[pos] = n_forced + j0 + i;
-    ++pos;
+#pragma unroll
+  for (int w = 0; w < (KPL > 64 ? 2 : 1); ++w) {
+    uint64_t take = w == 0 ? take0 : take1;
+    while (take != 0ull) {
+      const int i = __ffsll(static_cast<long long>(take)) - 1 + 64 * w;
+      take &= take - 1ull;
+      if (pos < K) ordered[pos] = n_forced + j0 + i;
+      ++pos;
+    }
   }
   __syncwarp();
   for (uint32_t p = lane; p < K; p += 32) out[n_forced + p] = ordered[p];
 }
 
-// One warp per row, kTopkWarps rows per CTA; grid.x = ceil(H * nqb / kTopkWarps). Requires
-// 1 <= k_topk < n_cand and n_cand + 3 <= 32 * KPL (room for the row's slot offset).
-constexpr int kTopkWarps = 4;
+// One warp per row, topk_cta_warps(KPL) rows per CTA (two for the longest rows, so that the
+// static shared memory stays under 48 KB); grid.x = ceil(H * nqb / topk_cta_warps(KPL)).
+// Requires 1 <= k_topk < n_cand and n_cand + 3 <= 32 * KPL (room for the row's slot offset).
+__host__ __device__ constexpr int topk_cta_warps(int kpl) { return kpl > 64 ? 2 : 4; }
 
 template <int KPL>
 struct TopkSmem {
-  alignas(16) float sv[kTopkWarps][32 * KPL];
-  uint32_t binw[kTopkWarps][8 * KPL];
-  uint32_t hist[kTopkWarps][256];
-  uint32_t gat[kTopkWarps][32];
+  static constexpr int kW = topk_cta_warps(KPL);
+  alignas(16) float sv[kW][32 * KPL];
+  uint32_t binw[kW][8 * KPL];
+  uint32_t hist[kW][256];
+  uint32_t gat[kW][32];
 };
 
 template <int KPL>
-__global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const float* __restrict__ S, int64_t rows,
-                                                                    int nkb, int n_forced, int k_topk,
-                                                                    int32_t* __restrict__ idx,
-                                                                    int32_t* __restrict__ cnt, int kmax) {
+__global__ void __launch_bounds__(32 * topk_cta_warps(KPL)) topk_warp_kernel(const float* __restrict__ S,
+                                                                             int64_t rows, int nkb, int n_forced,
+                                                                             int k_topk, int32_t* __restrict__ idx,
+                                                                             int32_t* __restrict__ cnt, int kmax) {
   __shared__ TopkSmem<KPL> sm;
   const int w = threadIdx.x >> 5;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kTopkWarps + w;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * topk_cta_warps(KPL) + w;
   griddep_wait();  // scores come from the preceding score kernel
   if (row >= rows) return;
   topk_row_warp<KPL>(S + row * nkb + n_forced, nkb - n_forced, n_forced, k_topk, idx + row * kmax, sm.sv[w],

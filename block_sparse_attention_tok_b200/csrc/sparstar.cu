@@ -171,36 +171,30 @@ cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
 // Keys per lane of the warp Top-K: the smallest supported count that covers n_cand
 // candidates, or 0 when the shared-memory radix kernel has to be used.
 int topk_keys_per_lane(int64_t n_cand) {
-  for (int kpl : {8, 16, 24, 36, 48, 64})
+  for (int kpl : {8, 16, 24, 36, 48, 64, 76, 124})
     if (n_cand <= 32 * kpl) return kpl;
   return 0;
 }
 
 // Top-K of `rows` score rows of nkb columns (1 <= k_topk < nkb - n_forced <= kMaxCandidates):
-// one warp per row up to 2045 candidates, else one CTA per row. Launched with programmatic
+// one warp per row up to 3965 candidates, else one CTA per row. Launched with programmatic
 // stream serialization, so it may start while a preceding score kernel drains.
 void launch_topk(const float* S, int64_t rows, int nkb, int n_forced, int k_topk, int32_t* idx, int32_t* cnt,
                  int kmax, cudaStream_t st) {
-  const dim3 wgrid(static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps)), wblock(32 * kTopkWarps);
+  auto warp_kernel = [&](auto kernel, int kpl) {
+    const int w = topk_cta_warps(kpl);
+    launch_after(kernel, dim3(static_cast<unsigned>((rows + w - 1) / w)), dim3(32 * w), 0, st, S, rows, nkb, n_forced,
+                 k_topk, idx, cnt, kmax);
+  };
   switch (topk_keys_per_lane(nkb - n_forced + 3)) {  // + the staging slot offset (<= 3)
-    case 8:
-      launch_after(topk_warp_kernel<8>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
-    case 16:
-      launch_after(topk_warp_kernel<16>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
-    case 24:
-      launch_after(topk_warp_kernel<24>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
-    case 36:
-      launch_after(topk_warp_kernel<36>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
-    case 48:
-      launch_after(topk_warp_kernel<48>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
-    case 64:
-      launch_after(topk_warp_kernel<64>, wgrid, wblock, 0, st, S, rows, nkb, n_forced, k_topk, idx, cnt, kmax);
-      break;
+    case 8: warp_kernel(topk_warp_kernel<8>, 8); break;
+    case 16: warp_kernel(topk_warp_kernel<16>, 16); break;
+    case 24: warp_kernel(topk_warp_kernel<24>, 24); break;
+    case 36: warp_kernel(topk_warp_kernel<36>, 36); break;
+    case 48: warp_kernel(topk_warp_kernel<48>, 48); break;
+    case 64: warp_kernel(topk_warp_kernel<64>, 64); break;
+    case 76: warp_kernel(topk_warp_kernel<76>, 76); break;
+    case 124: warp_kernel(topk_warp_kernel<124>, 124); break;
     default:
       launch_after(topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(128),
                    static_cast<size_t>(nkb - n_forced) * 4, st, S, nkb, n_forced, k_topk, idx, cnt, kmax);

@@ -3,7 +3,7 @@ run with block = 64: masks by the same gap rule, outputs element by element.
 
 With 64-token blocks a query block is 64 rows of the kernel's 128-row MMA tile (the other
 64 rows are computed and dropped), a KV tile is one 64-token block, and rows with more than
-2,045 candidates go through the radix Top-K.
+3,965 candidates go through the radix Top-K.
 """
 import math
 
@@ -73,11 +73,11 @@ def test_block64_small_cases(S, d, n_q, n_text, n_ctx, n_cur, clip, density):
 
 
 def test_block64_radix_topk_rows(S):
-    """More than 2,045 candidates per row: the CTA-per-row radix Top-K path."""
-    n_cur = 64 * 2100
+    """More than 3,965 candidates per row: the CTA-per-row radix Top-K path."""
+    n_cur = 64 * 4000
     q, k, v = synth.make_qkv(200, 64 + n_cur, 1, 128, [811], device="cuda")
     stats, plan = _run(S, q, k, v, 64, 0, n_cur, 2, 0.05, qblocks=lambda n: [0, n - 1])
-    assert int(plan.n_cand) > 2045 and stats["rows"] == int(plan.nqb)
+    assert int(plan.n_cand) > 3965 and stats["rows"] == int(plan.nqb)
 
 
 @pytest.mark.parametrize("d", [64, 128])

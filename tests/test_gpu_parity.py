@@ -266,10 +266,10 @@ def test_schedule_scales(S, scale_index, layer):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("n_cand", [2045, 2046])
+@pytest.mark.parametrize("n_cand", [3965, 3966])
 def test_topk_path_boundary(S, n_cand):
-    """2,045 candidates is the largest row the warp Top-K takes (64 keys per lane, 3 slots kept
-    for the row's alignment offset); 2,046 goes to the CTA-per-row radix Top-K. Both must give
+    """3,965 candidates is the largest row the warp Top-K takes (124 keys per lane, 3 slots kept
+    for the row's alignment offset); 3,966 goes to the CTA-per-row radix Top-K. Both must give
     the oracle's masks."""
     n_text, n_q = 128, 256
     q, k, v = synth.make_qkv(n_q, n_text + 128 * n_cand, 1, 64, [4000 + n_cand], device="cuda")

@@ -7,7 +7,7 @@ of the kernels: ordinary rows; heavy ties (small integers), so that equal scores
 the K-th place; constant rows; signed zeros; NaN, sparse and dominant (K beyond the count of
 numbers); infinities; an outlier that squeezes every other score into one value bin; a
 denormal-width range; a range wider than the largest float. Sizes cover every keys-per-lane
-instance of the warp kernel, the 2,045-candidate boundary to the CTA-per-row kernel, and
+instance of the warp kernel, the 3,965-candidate boundary to the CTA-per-row kernel, and
 the rows that never read scores (K_topk = 0 or every candidate kept).
 """
 import numpy as np
@@ -85,7 +85,7 @@ def _check(S_lib, s32, n_forced, k_topk, kmax=None):
 
 
 @pytest.mark.parametrize("kind", KINDS)
-@pytest.mark.parametrize("n_cand", [2, 33, 256, 257, 700, 1128, 1153, 1600, 2045, 2046, 5000])
+@pytest.mark.parametrize("n_cand", [2, 33, 256, 257, 700, 1128, 1153, 1600, 2045, 2046, 2256, 3100, 3965, 3966, 5000])
 def test_topk_matches_oracle(S, kind, n_cand):
     rng = np.random.default_rng(100003 * KINDS.index(kind) + n_cand)
     n_forced = int(rng.integers(0, 6))
@@ -96,7 +96,7 @@ def test_topk_matches_oracle(S, kind, n_cand):
             _check(S, s, n_forced, k_topk)
 
 
-@pytest.mark.parametrize("kpl_edge", [253, 509, 765, 1149, 1533, 2045])
+@pytest.mark.parametrize("kpl_edge", [253, 509, 765, 1149, 1533, 2045, 2429, 3965])
 def test_topk_keys_per_lane_edges(S, kpl_edge):
     """The largest row of each warp kernel instance (32 * keys per lane, less 3 slots for the
     row's 16-byte alignment offset), and one candidate more."""
