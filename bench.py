@@ -455,8 +455,9 @@ def run_ours(args, rank, world, local_rank):
             "attn_ms": t_att64, "attn_tflops": flops64 / (t_att64 * 1e-3) / 1e12,
             "kept_tile_tflop": flops64 / 1e12, "select_us": t_sel64 * 1e3,
             "select_gbs": sel_bytes64 / (t_sel64 * 1e-3) / 1e9, "step_ms": t_sel64 + t_att64,
-            "note": "64-row query blocks run as half of a 128-row MMA tile and 64-token KV tiles use "
-                    "N = 64 MMAs, so per kept FLOP the tensor cores do about 2x the work of block 128"}
+            "note": "64-row query blocks run as half of a 128-row MMA tile (pairs of kept 64-token KV "
+                    "blocks form one 128-token tile), so per kept FLOP the tensor cores do about 2x the "
+                    "work of block 128"}
         del ws64, idx64, cnt64, o64
         torch.cuda.empty_cache()
 

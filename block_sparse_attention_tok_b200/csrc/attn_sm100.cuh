@@ -36,21 +36,26 @@
 namespace sparstar {
 
 // B = block size of the partition (128, or 64 for the block-size variant): a query block is B
-// rows of the 128-row MMA tile (with B = 64 the other 64 rows are computed and dropped) and a
-// KV tile is one B-token KV block (MMA N = B for QK^T, K = B for PV).
+// rows of the 128-row MMA tile (with B = 64 the other 64 rows are computed and dropped), and a
+// KV tile is 128 tokens: one KV block, or with B = 64 two consecutive entries of the kept
+// list, each loaded as its own 64-row box into one half of the stage (a 64-row box at a
+// 1 KB-aligned offset lands in the same swizzled layout as rows 64-127 of a 128-row box).
+// An odd last entry fills both halves with the same block and the second half is masked.
 template <int D, int B = 128>
 struct AttnConfig {
   static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
   static_assert(B == 64 || B == 128, "block must be 64 or 128");
   static constexpr int kRows = 128;                    // query rows per MMA tile
-  static constexpr int kCols = B;                      // KV tokens per tile (one KV block)
-  static constexpr int kSC = B / 32;                   // 32-column chunks of an S row
+  static constexpr int kCols = 128;                    // KV tokens per tile
+  static constexpr int kBlocksPerTile = kCols / B;     // KV blocks per tile
+  static constexpr int kSC = kCols / 32;               // 32-column chunks of an S row
   static constexpr int kChunks = D / 64;               // 128-byte swizzle chunks per row
   static constexpr uint32_t kQChunkBytes = 128 * 128;  // 128 rows x 128 bytes
-  static constexpr uint32_t kKVChunkBytes = B * 128;   // B rows x 128 bytes
+  static constexpr uint32_t kKVChunkBytes = kCols * 128;  // 128 rows x 128 bytes
+  static constexpr uint32_t kKVBoxBytes = B * 128;     // one KV block's rows of a chunk
   static constexpr uint32_t kQTileBytes = kChunks * kQChunkBytes;
   static constexpr uint32_t kKVTileBytes = kChunks * kKVChunkBytes;
-  static constexpr int kStages = ((D == 128) ? 4 : 8) * (128 / B);  // K/V ring depth
+  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth
   static constexpr int kSlots = 2;
   static constexpr int kThreads = 320;                 // 8 softmax warps + TMA warp + MMA warp
   static constexpr int kLoadWarp = 8;
@@ -59,7 +64,7 @@ struct AttnConfig {
   static constexpr uint32_t kTmemS = 0;                // + 128 * slot
   static constexpr uint32_t kTmemO = 256;              // + 128 * slot
   static constexpr uint32_t kSmemBytes = 1024 /*align*/ + kSlots * kQTileBytes + kStages * kKVTileBytes + 512;
-  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, B, false);
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kCols, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
 };
 
@@ -77,7 +82,8 @@ struct AttnParams {
 // Work sequence of one slot: items slot_id, slot_id + stride, ... (head-major order).
 struct SlotSeq {
   int item;     // current item, or -1 when the slot is finished
-  int ntiles;   // kept blocks of the current item
+  int nblk;     // kept blocks of the current item
+  int ntiles;   // tiles of the current item (kept blocks / blocks per tile, rounded up)
   int n;        // current tile within the item
   int k;        // number of items started before the current one
   int h, qb;
@@ -99,6 +105,7 @@ __device__ __forceinline__ int clamp_block(int j, int nkb, unsigned* status, boo
   return j;
 }
 
+template <int BPT>
 __device__ __forceinline__ void seq_begin(SlotSeq& s, const AttnParams& p, bool report) {
   if (s.item >= p.n_items) {
     s.item = -1;
@@ -106,27 +113,35 @@ __device__ __forceinline__ void seq_begin(SlotSeq& s, const AttnParams& p, bool 
   }
   s.h = s.item / p.nqb;
   s.qb = s.item - s.h * p.nqb;
-  s.ntiles = clamp_count(__ldg(p.cnt + s.item), p.kmax, p.status, report);
+  s.nblk = clamp_count(__ldg(p.cnt + s.item), p.kmax, p.status, report);
+  s.ntiles = BPT == 1 ? s.nblk : (s.nblk + BPT - 1) / BPT;
   s.n = 0;
 }
 
+template <int BPT>
 __device__ __forceinline__ void seq_init(SlotSeq& s, int slot_id, const AttnParams& p, bool report) {
   s.item = slot_id;
   s.k = 0;
-  seq_begin(s, p, report);
+  seq_begin<BPT>(s, p, report);
 }
 
 // Advance to the next tile; returns true when a new item started.
+template <int BPT>
 __device__ __forceinline__ bool seq_next(SlotSeq& s, int stride, const AttnParams& p, bool report) {
   if (++s.n < s.ntiles) return false;
   s.item += stride;
   ++s.k;
-  seq_begin(s, p, report);
+  seq_begin<BPT>(s, p, report);
   return true;
 }
 
-__device__ __forceinline__ int seq_block(const SlotSeq& s, const AttnParams& p, bool report) {
-  const int j = __ldg(p.idx + static_cast<int64_t>(s.item) * p.kmax + s.n);
+// KV block of part `half` of the current tile; a part past the end of the kept list (the odd
+// last entry with two blocks per tile) repeats the tile's first block.
+template <int BPT>
+__device__ __forceinline__ int seq_block(const SlotSeq& s, const AttnParams& p, bool report, int half = 0) {
+  int e = s.n * BPT + half;
+  if (BPT > 1 && e >= s.nblk) e = s.n * BPT;
+  const int j = __ldg(p.idx + static_cast<int64_t>(s.item) * p.kmax + e);
   return clamp_block(j, p.nkb, p.status, report);
 }
 
@@ -184,7 +199,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     attn_sparse_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnConfig<D, B>;
-  static_assert(kPolyCols % 32 == 0 && kPolyCols <= B, "software exp2 works on whole 32-column chunks");
+  static_assert(kPolyCols % 32 == 0 && kPolyCols <= C::kCols, "software exp2 works on whole 32-column chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -241,8 +256,8 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       SlotSeq seq0, seq1;
-      seq_init(seq0, blockIdx.x * 2 + 0, p, true);
-      seq_init(seq1, blockIdx.x * 2 + 1, p, true);
+      seq_init<C::kBlocksPerTile>(seq0, blockIdx.x * 2 + 0, p, true);
+      seq_init<C::kBlocksPerTile>(seq1, blockIdx.x * 2 + 1, p, true);
       uint32_t ring_it = 0;
       int last_q_k0 = -1, last_q_k1 = -1;
       bool ok = true;
@@ -258,7 +273,9 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         return true;
       };
       auto load_kv = [&](SlotSeq& sq, const CUtensorMap* map) -> bool {
-        const int j = seq_block(sq, p, true);
+        int jb[C::kBlocksPerTile];
+#pragma unroll
+        for (int b = 0; b < C::kBlocksPerTile; ++b) jb[b] = seq_block<C::kBlocksPerTile>(sq, p, true, b);
         const uint32_t stage = ring_it % C::kStages;
         const uint32_t phase = (ring_it / C::kStages) & 1u;
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) return false;
@@ -266,7 +283,9 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         const uint32_t dst = smem_u32(ring + stage * C::kKVTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kKVChunkBytes, map, &full[stage], c * 64, j * B, sq.h);
+#pragma unroll
+          for (int b = 0; b < C::kBlocksPerTile; ++b)
+            tma_load_3d(dst + c * C::kKVChunkBytes + b * C::kKVBoxBytes, map, &full[stage], c * 64, jb[b] * B, sq.h);
         ++ring_it;
         return true;
       };
@@ -275,7 +294,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         if (!ok || sq.item < 0) return;
         ok = load_kv(sq, &tm_v);
         if (!ok) return;
-        const bool new_item = seq_next(sq, stride, p, true);
+        const bool new_item = seq_next<C::kBlocksPerTile>(sq, stride, p, true);
         if (sq.item < 0) return;
         if (new_item) ok = load_q(s, sq, last_k);
         if (ok) ok = load_kv(sq, &tm_k);
@@ -313,8 +332,8 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     // and descriptors stay in uniform registers); one elected lane issues each batch of
     // tcgen05.mma / tcgen05.commit. Issue cost, not tensor time, bounds a lane-0-only loop.
     SlotSeq seq0, seq1;
-    seq_init(seq0, blockIdx.x * 2 + 0, p, false);
-    seq_init(seq1, blockIdx.x * 2 + 1, p, false);
+    seq_init<C::kBlocksPerTile>(seq0, blockIdx.x * 2 + 0, p, false);
+    seq_init<C::kBlocksPerTile>(seq1, blockIdx.x * 2 + 1, p, false);
     uint32_t ring_it = 0;
     uint32_t tiles0 = 0u, tiles1 = 0u;
     bool ok = true;
@@ -362,9 +381,9 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
       const uint32_t a_tmem = tmem_base + C::kTmemS + 128u * s;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < B / 16; ++kk) {
+        for (int kk = 0; kk < C::kCols / 16; ++kk) {
           // P columns: 16 bf16 per K step = 8 packed 32-bit columns.
-          // V tile is MN-major for this MMA: 64-element chunks of d at B*128 bytes (LBO),
+          // V tile is MN-major for this MMA: 64-element chunks of d at 128*128 bytes (LBO),
           // 8-row groups of KV tokens at 1 KB (SBO); a K step of 16 tokens advances 2 KB.
           mma_ts(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), C::kIdescPV, (sq.n > 0 || kk > 0) ? 1u : 0u);
         }
@@ -380,7 +399,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
       if (!ok || sq.item < 0) return;
       ok = issue_pv(s, sq, tiles);
       if (!ok) return;
-      seq_next(sq, stride, p, false);
+      seq_next<C::kBlocksPerTile>(sq, stride, p, false);
       if (sq.item < 0) return;
       ok = issue_s(s, sq);
     };
@@ -408,15 +427,24 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     const uint32_t t_o = tmem_base + lane_off + C::kTmemO + 128u * s;
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     SlotSeq seq;
-    seq_init(seq, blockIdx.x * 2 + s, p, false);
+    seq_init<C::kBlocksPerTile>(seq, blockIdx.x * 2 + s, p, false);
     uint32_t tiles = 0, items = 0;
     bool ok = true;
     while (ok && seq.item >= 0) {
       float m_run = -INFINITY, l_run = 0.f;
       for (int n = 0; n < seq.ntiles && ok; ++n) {
         seq.n = n;
-        const int j = seq_block(seq, p, false);
-        const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * B) : B;
+        // valid columns of each part of the tile (a ragged last KV block; 0 for the repeated
+        // half of an odd last entry)
+        int n_valid[C::kBlocksPerTile];
+        bool ragged = false;
+#pragma unroll
+        for (int b = 0; b < C::kBlocksPerTile; ++b) {
+          const int j = seq_block<C::kBlocksPerTile>(seq, p, false, b);
+          n_valid[b] = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * B) : B;
+          if (b > 0 && n * C::kBlocksPerTile + b >= seq.nblk) n_valid[b] = 0;
+          ragged |= n_valid[b] < B;
+        }
         // tcgen05.ld/st below are warp-collective: every lane must take the same path.
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], tiles & 1u, abort_flag, p.status))) {
           ok = false;
@@ -428,12 +456,12 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < C::kSC; ++c) tmem_ld32(t_s + 32 * c, r[c]);
         tmem_wait_ld();
-        if (n_valid < B) {
+        if (ragged) {
 #pragma unroll
           for (int c = 0; c < C::kSC; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (32 * c + e >= n_valid) r[c][e] = __float_as_uint(-INFINITY);
+              if ((32 * c + e) % B >= n_valid[(32 * c + e) / B]) r[c][e] = __float_as_uint(-INFINITY);
         }
         const float mx_scaled = row_max<C::kSC>(r) * p.scale_log2;
         float alpha = 1.f;
@@ -482,7 +510,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
             tmem_st32(t_o + 32 * c, ov);
           }
         }
-        // P: B bf16 = B/2 packed columns over the start of S.
+        // P: kCols bf16 = kCols/2 packed columns over the start of S.
 #pragma unroll
         for (int c = 0; c < C::kSC / 2; ++c) {
           uint32_t pk[32];
@@ -526,7 +554,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         p.lse[static_cast<int64_t>(seq.h) * p.n_q + t] = (m_run + log2f(l_run)) * 0.6931471805599453f;
       tc_fence_before();
       seq.n = seq.ntiles - 1;
-      seq_next(seq, stride, p, false);
+      seq_next<C::kBlocksPerTile>(seq, stride, p, false);
     }
   }
 

@@ -2,8 +2,9 @@
 run with block = 64: masks by the same gap rule, outputs element by element.
 
 With 64-token blocks a query block is 64 rows of the kernel's 128-row MMA tile (the other
-64 rows are computed and dropped), a KV tile is one 64-token block, and rows with more than
-3,965 candidates go through the radix Top-K.
+64 rows are computed and dropped), a KV tile is two consecutive kept 64-token blocks (an odd
+last one alone, its second half masked), and rows with more than 3,965 candidates go
+through the radix Top-K.
 """
 import math
 
@@ -88,6 +89,31 @@ def test_block64_attention_on_random_masks(S, d, n_q, n_kv):
     rng = np.random.default_rng(n_q * 7 + n_kv)
     kk = max(1, min(nkb, int(rng.integers(1, nkb + 1))))
     rows = np.stack([np.stack([np.sort(rng.choice(nkb, kk, replace=False)) for _ in range(nqb)]) for _ in range(2)])
+    idx = torch.from_numpy(rows.astype(np.int32)).cuda().contiguous()
+    cnt = torch.full((2, nqb), kk, dtype=torch.int32, device="cuda")
+    o, lse = S.attn(q, k, v, idx, cnt, block=B)
+    assert S.device_status() == S.OK
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(2):
+        outs = O.block_sparse_attention(_f64(qb[h]), _f64(kb[h]), _f64(vb[h]), rows[h], range(nqb), block=B)
+        for i, (o_ref, lse_ref) in enumerate(outs):
+            s, e = O.block_token_range(i, n_q, B)
+            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
+            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("kk", [1, 2, 3, 4, 7, 10])
+def test_block64_pairs_odd_even_and_ragged(S, kk):
+    """Kept lists of odd and even length, each ending with the ragged last KV block (17 valid
+    tokens): it is then the second half of a pair (even length) or the lone last entry (odd),
+    and the lists mix adjacent and distant blocks, so pairs are not contiguous in memory."""
+    d, n_q, n_kv = 128, 130, 64 * 9 + 17
+    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [31 + kk, 41 + kk], device="cuda")
+    nqb, nkb = O.num_blocks(n_q, B), O.num_blocks(n_kv, B)
+    rng = np.random.default_rng(900 + kk)
+    rows = np.stack([np.stack([np.sort(np.append(rng.choice(nkb - 1, kk - 1, replace=False), nkb - 1))
+                               for _ in range(nqb)]) for _ in range(2)])
     idx = torch.from_numpy(rows.astype(np.int32)).cuda().contiguous()
     cnt = torch.full((2, nqb), kk, dtype=torch.int32, device="cuda")
     o, lse = S.attn(q, k, v, idx, cnt, block=B)
