@@ -103,13 +103,14 @@ def test_block64_attention_on_random_masks(S, d, n_q, n_kv):
             assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("kk", [1, 2, 3, 4, 7, 10])
-def test_block64_pairs_odd_even_and_ragged(S, kk):
+def test_block64_pairs_odd_even_and_ragged(S, d, kk):
     """Kept lists of odd and even length, each ending with the ragged last KV block (17 valid
     tokens): it is then the second half of a pair (even length) or the lone last entry (odd),
     and the lists mix adjacent and distant blocks, so pairs are not contiguous in memory."""
-    d, n_q, n_kv = 128, 130, 64 * 9 + 17
-    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [31 + kk, 41 + kk], device="cuda")
+    n_q, n_kv = 130, 64 * 9 + 17
+    q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [31 + kk + d, 41 + kk + d], device="cuda")
     nqb, nkb = O.num_blocks(n_q, B), O.num_blocks(n_kv, B)
     rng = np.random.default_rng(900 + kk)
     rows = np.stack([np.stack([np.sort(np.append(rng.choice(nkb - 1, kk - 1, replace=False), nkb - 1))
