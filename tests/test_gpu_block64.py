@@ -108,14 +108,18 @@ def test_block64_attention_on_random_masks(S, d, n_q, n_kv):
 def test_block64_pairs_odd_even_and_ragged(S, d, kk):
     """Kept lists of odd and even length, each ending with the ragged last KV block (17 valid
     tokens): it is then the second half of a pair (even length) or the lone last entry (odd),
-    and the lists mix adjacent and distant blocks, so pairs are not contiguous in memory."""
+    and the lists mix adjacent and distant blocks, so pairs are not contiguous in memory. The
+    index rows are wider than cnt, so an odd list's missing partner is never read."""
     n_q, n_kv = 130, 64 * 9 + 17
     q, k, v = synth.make_qkv(n_q, n_kv, 2, d, [31 + kk + d, 41 + kk + d], device="cuda")
     nqb, nkb = O.num_blocks(n_q, B), O.num_blocks(n_kv, B)
     rng = np.random.default_rng(900 + kk)
     rows = np.stack([np.stack([np.sort(np.append(rng.choice(nkb - 1, kk - 1, replace=False), nkb - 1))
                                for _ in range(nqb)]) for _ in range(2)])
-    idx = torch.from_numpy(rows.astype(np.int32)).cuda().contiguous()
+    # entries past cnt hold an out-of-range block: reading one would raise the bounds flag
+    padded = np.full((2, nqb, kk + 3), -7, dtype=np.int32)
+    padded[:, :, :kk] = rows
+    idx = torch.from_numpy(padded).cuda().contiguous()
     cnt = torch.full((2, nqb), kk, dtype=torch.int32, device="cuda")
     o, lse = S.attn(q, k, v, idx, cnt, block=B)
     assert S.device_status() == S.OK
