@@ -12,6 +12,8 @@
 //     and V tiles into a ring of shared-memory stages (128-byte swizzle; each CTA loads its own);
 //   * warp 9 (MMA, one thread): S = Q K^T into tensor memory (tcgen05.mma, M=128, N=128,
 //     K=16 steps), then O += P V with P read from tensor memory;
+//   * warps 10-11: idle, they complete the producer warpgroup so that setmaxnreg can move
+//     its registers to the softmax warps;
 //   * warps 0-3 / 4-7 (softmax of slot 0 / 1, one thread per query row): tcgen05.ld of the
 //     S row, masking of a ragged last KV block, running max with a lazy rescale (the
 //     running max only moves when a tile's max exceeds it by more than 8 in log2 units,
@@ -57,7 +59,16 @@ struct AttnConfig {
   static constexpr uint32_t kKVTileBytes = kChunks * kKVChunkBytes;
   static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth
   static constexpr int kSlots = 2;
-  static constexpr int kThreads = 320;                 // 8 softmax warps + TMA warp + MMA warp
+  // 8 softmax warps (warpgroups 0 and 1), then the producer warpgroup: TMA warp, MMA warp and
+  // two idle warps. Three warps share each SM sub-partition's 16 K-register file, so the block
+  // launches at 168 registers a thread; setmaxnreg then moves registers from the producer
+  // warpgroup (whose code needs 76) to the softmax warpgroups, which would spill at 168.
+  static constexpr int kThreads = 384;
+  static constexpr int kLaunchRegs = (65536 / kThreads) & ~7;  // 168
+  static constexpr int kRegsSoftmax = 208;             // per thread, warpgroups 0 and 1
+  static constexpr int kRegsProducer = 80;             // per thread, warpgroup 2
+  static constexpr int kRegsNeeded = 256 * kRegsSoftmax + 128 * kRegsProducer;
+  static_assert(kRegsNeeded <= kThreads * kLaunchRegs, "setmaxnreg split above the launch allocation");
   static constexpr int kLoadWarp = 8;
   static constexpr int kMmaWarp = 9;
   static constexpr uint32_t kTmemCols = 512;
@@ -252,6 +263,10 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Each role lowers or raises its register count inside its own branch (a count changed
+  // before a merge point would bind the code after it for every warp).
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegsProducer));
   if (warp == C::kLoadWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -417,7 +432,9 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
     }
     __syncwarp();
+  }  // warps 10 and 11 only complete the warpgroup
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegsSoftmax));
     // ------------------------------------------------------------ softmax / epilogue
     const int s = warp >> 2;          // slot
     const int wq = warp & 3;          // TMEM lane quarter

@@ -113,6 +113,18 @@ int set_kernel_attrs(DeviceInfo* d) {
   ok &= cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMaxCandidates * 4)) == cudaSuccess;
   if (!ok) return SPARSTAR_ERR_CUDA;
+  // The attention kernels raise the softmax warps' registers with setmaxnreg, drawing on the
+  // block's launch allocation; a build that launched with fewer registers would wait there
+  // for good, so such a build is refused before any launch.
+  auto regs_ok = [](auto kernel, int threads, int needed) {
+    cudaFuncAttributes a;
+    return cudaFuncGetAttributes(&a, kernel) == cudaSuccess && a.numRegs * threads >= needed;
+  };
+  if (!regs_ok(attn_sparse_kernel<128, kPolyCols128>, AttnConfig<128>::kThreads, AttnConfig<128>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<64, kPolyCols64>, AttnConfig<64>::kThreads, AttnConfig<64>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<128, 0, 64>, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<64, 0, 64>, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kRegsNeeded))
+    return SPARSTAR_ERR_UNSUPPORTED;
   d->attrs_set = true;
   return SPARSTAR_OK;
 }
