@@ -9,7 +9,9 @@
 //     sequence of (head, query block) items, so the softmax of one slot overlaps the tensor
 //     core work of the other;
 //   * warp 8 (TMA): loads the slot's 128xd Q tile once per item and, per kept block, the K
-//     and V tiles into a ring of shared-memory stages (128-byte swizzle; each CTA loads its own);
+//     and V tiles into a ring of shared-memory stages (128-byte swizzle; each CTA loads its own;
+//     Q with an L2 evict-first policy, K/V evict-last, and O is written with streaming stores,
+//     so that the K/V of the head in flight stays in L2);
 //   * warp 9 (MMA, one thread): S = Q K^T into tensor memory (tcgen05.mma, M=128, N=128,
 //     K=16 steps), then O += P V with P read from tensor memory;
 //   * warps 10-11: idle, they complete the producer warpgroup so that setmaxnreg can move
@@ -276,6 +278,9 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
       uint32_t ring_it = 0;
       int last_q_k0 = -1, last_q_k1 = -1;
       bool ok = true;
+      // Q is read once per item: evicted first. K/V of the current head is re-read by every
+      // query block that keeps it: kept last.
+      const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
 
       auto load_q = [&](int s, SlotSeq& sq, int& last_k) -> bool {
         if (!mbar_wait(&q_empty[s], (sq.k & 1) ^ 1, abort_flag, p.status)) return false;
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         const uint32_t dst = smem_u32(q_tile + s * C::kQTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kQChunkBytes, &tm_q, &q_full[s], c * 64, sq.qb * B, sq.h);
+          tma_load_3d_hint(dst + c * C::kQChunkBytes, &tm_q, &q_full[s], c * 64, sq.qb * B, sq.h, pol_q);
         last_k = sq.k;
         return true;
       };
@@ -300,7 +305,8 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
           for (int b = 0; b < C::kBlocksPerTile; ++b)
-            tma_load_3d(dst + c * C::kKVChunkBytes + b * C::kKVBoxBytes, map, &full[stage], c * 64, jb[b] * B, sq.h);
+            tma_load_3d_hint(dst + c * C::kKVChunkBytes + b * C::kKVBoxBytes, map, &full[stage], c * 64, jb[b] * B,
+                             sq.h, pol_kv);
         ++ring_it;
         return true;
       };
@@ -564,11 +570,11 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            __stcs(dst + v4, make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]));
         }
       }
       if (valid && p.lse != nullptr)
-        p.lse[static_cast<int64_t>(seq.h) * p.n_q + t] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+        __stcs(p.lse + static_cast<int64_t>(seq.h) * p.n_q + t, (m_run + log2f(l_run)) * 0.6931471805599453f);
       tc_fence_before();
       seq.n = seq.ntiles - 1;
       seq_next<C::kBlocksPerTile>(seq, stride, p, false);
