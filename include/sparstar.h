@@ -54,7 +54,9 @@ extern "C" {
 /* Return codes. */
 #define SPARSTAR_OK 0
 #define SPARSTAR_ERR_ARG 1             /* bad pointer, size, alignment, density or clip */
-#define SPARSTAR_ERR_UNSUPPORTED 2     /* head_dim not in {64,128}, device not sm_100, size beyond a limit */
+#define SPARSTAR_ERR_UNSUPPORTED 2     /* head_dim not in {64,128}, device not sm_100, size beyond a limit,
+                                         or a library build whose attention kernels launch with
+                                         too few registers for their setmaxnreg split */
 #define SPARSTAR_ERR_WORKSPACE 3       /* workspace NULL or smaller than sparstar_workspace_size() */
 #define SPARSTAR_ERR_CUDA 4            /* a CUDA runtime/driver call failed */
 #define SPARSTAR_ERR_DEVICE_TIMEOUT 5  /* a kernel's bounded wait expired (reported by sparstar_device_status) */
