@@ -47,3 +47,15 @@ def test_attention_is_bitwise_reproducible_into_the_same_buffers(S):
     S.attn(q, k, v, idx, cnt, o=o, lse=lse)
     assert S.device_status() == S.OK
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+def test_attention_without_lse_gives_the_same_output(S):
+    """With no LSE buffer (a null pointer through the C ABI) the kernel skips that store only."""
+    n_text, n_ctx, n_cur = 128, 2048, 3000
+    q, k, v = synth.make_qkv(n_cur, n_text + n_ctx + n_cur, 2, 128, [81, 82], device="cuda")
+    idx, cnt, _ = S.select(q, k, n_text, n_ctx, n_cur, 2, 0.2)
+    o_with, lse = S.attn(q, k, v, idx, cnt)
+    o_without, none = S.attn(q, k, v, idx, cnt, want_lse=False)
+    assert S.device_status() == S.OK
+    assert none is None and lse is not None
+    assert torch.equal(o_with, o_without)
