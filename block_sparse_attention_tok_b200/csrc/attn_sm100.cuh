@@ -518,6 +518,17 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[c][e] = pk[e];
+          if (c & 1) {
+            // P: kCols bf16 = kCols/2 packed columns over the start of S; each 32-column
+            // store leaves as soon as its two chunks are done (one wait for all at the end)
+            uint32_t p32[32];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              p32[e] = r[c - 1][e];
+              p32[16 + e] = r[c][e];
+            }
+            tmem_st32(t_s + 16 * (c - 1), p32);
+          }
         }
         const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
         const float2 a = __fadd2_rn(a01, a23);
@@ -532,17 +543,6 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
             tmem_st32(t_o + 32 * c, ov);
           }
-        }
-        // P: kCols bf16 = kCols/2 packed columns over the start of S.
-#pragma unroll
-        for (int c = 0; c < C::kSC / 2; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            pk[e] = r[2 * c][e];
-            pk[16 + e] = r[2 * c + 1][e];
-          }
-          tmem_st32(t_s + 32 * c, pk);
         }
         tmem_wait_st();
         tc_fence_before();
