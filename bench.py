@@ -4,11 +4,17 @@ A step is the whole per-scale path (pooling, scores, Top-K, attention over the k
 over one 720p final-scale Clip-2 input (32 heads, d 128, 72,192 query tokens, KV 512 text +
 72,192 preceding-clip + 72,192 current tokens, density 0.09375), inputs resident in HBM.
 
+With N GPUs (one process per GPU, NCCL for the barrier and the timing reduction only) the
+default is strong scaling: rank r owns heads [r*H/N, (r+1)*H/N) of the one input and runs the
+path on them, with no collective on the path (heads are independent). `--scaling weak`
+instead gives every rank its own full scale. Without a torchrun environment, `--gpus N > 1`
+starts its own N ranks.
+
 Prints one JSON line (rank 0). Timed region: barrier + synchronize, K steps bracketed by
 CUDA events on the launch stream, synchronize + barrier; the max over ranks is reported.
-Inputs (3.5 GB per GPU) are far larger than L2 (126 MB), so no flush is inserted.
+Inputs (3.5 GB in total) are far larger than L2 (126 MB), so no flush is inserted.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--scaling strong|weak]
 """
 from __future__ import annotations
 
@@ -32,6 +38,7 @@ if ROOT not in sys.path:
 from block_sparse_attention_tok_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HBM_SPEC_GBS = 7700.0   # HGX B200 nominal HBM3e bandwidth
 METRIC = "sparse-attn TFLOP/s on kept tiles & % of bf16 peak; select GB/s; µs per scale"
 
 
@@ -41,6 +48,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--scaling", choices=["strong", "weak"], default="strong",
+                    help="strong: the ranks split the heads of one input; weak: every rank runs a full scale")
+    ap.add_argument("--gather-o", action="store_true",
+                    help="N > 1: also time one all-gather of O across ranks (outside the step)")
     ap.add_argument("--workload", default=synth.FINAL_CLIP2.name, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget-mode", type=int, default=0)
     ap.add_argument("--heads", type=int, default=0, help="limit the heads (profiling small cases); 0 = all")
@@ -168,8 +179,18 @@ def kept_tile_flops(idx: torch.Tensor, cnt: torch.Tensor, n_q: int, n_kv: int, d
 # ----------------------------------------------------------------------------- ranks
 
 def rank_seeds(sc, rank: int):
-    """Seeds of one rank's heads: every rank works on its own full scale (weak scaling)."""
+    """Seeds of one rank's heads under weak scaling: every rank works on its own full scale."""
     return [1000 * synth.CFG_INDEX.get(sc.name, 0) + h + 100000 * rank for h in range(sc.heads)]
+
+
+def sum_over_ranks(value: float, device, world: int) -> float:
+    """Sum of a per-rank quantity (a no-op on one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 def max_over_ranks(values, device, world: int):
@@ -182,9 +203,28 @@ def max_over_ranks(values, device, world: int):
     return [float(x) for x in t.tolist()]
 
 
-def whole_job_tflops(flops_per_rank: float, ms_max: float, world: int) -> float:
+def whole_job_tflops(flops_all_ranks: float, ms_max: float) -> float:
     """Aggregate throughput: the units all ranks processed over the slowest rank's time."""
-    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+    return flops_all_ranks / (ms_max * 1e-3) / 1e12
+
+
+def read_bandwidth_probe(dev, nbytes: int = 4 << 30, reps: int = 5) -> float:
+    """Best read-only streaming rate (GB/s) of a plain reduction over a buffer far larger than L2
+    (torch.sum of fp32 zeros, CUDA events): the denominator for read-only kernels such as the
+    selection, whose traffic is almost all reads, next to the copy figure (read + write)."""
+    x = torch.zeros(nbytes // 4, dtype=torch.float32, device=dev)
+    torch.sum(x)
+    best = 0.0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.sum(x)
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del x
+    torch.cuda.empty_cache()
+    return best
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -253,8 +293,8 @@ def run_reference(args, rank):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": float(np.mean(times) * 1e3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(sc, args), "impl": "reference",
+        "scaling": args.scaling, "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(sc, args, 1), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -262,12 +302,18 @@ def run_reference(args, rank):
     return 0
 
 
-def workload_config(sc, args):
+def workload_config(sc, args, world):
+    if args.scaling == "strong":
+        per_gpu = f"heads [r*{sc.heads}/{world}, (r+1)*{sc.heads}/{world}) of one input per rank r, no collective on the path"
+        par = f"heads/{world}"
+    else:
+        per_gpu = "one full scale (all heads) per rank"
+        par = f"replicas x{world}"
     return {"workload": sc.name, "heads": sc.heads, "head_dim": sc.head_dim, "n_q": sc.n_q,
             "kv": {"text": sc.n_text, "ctx": sc.n_ctx, "cur": sc.n_cur}, "clip": sc.clip,
             "density": sc.density, "budget": "literal" if args.budget_mode == 0 else "candidates",
-            "block": 128, "per_gpu": "one full scale (all heads) per rank",
-            "l2": "no flush: inputs 3.5 GB per GPU > 126 MB L2", "parallelism": f"replicas x{args.gpus}"}
+            "block": 128, "per_gpu": per_gpu,
+            "l2": "no flush: inputs 3.5 GB > 126 MB L2", "parallelism": par}
 
 
 def run_schedule(S, dev, stream, layers: int = 36):
@@ -340,10 +386,21 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     S.load()
-    sc = synth.WORKLOADS[args.workload]
+    from block_sparse_attention_tok_b200 import shard
+    sc_full = synth.WORKLOADS[args.workload]
     if args.heads:
-        sc = dataclasses.replace(sc, heads=args.heads)
-    q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim, rank_seeds(sc, rank), device=dev)
+        sc_full = dataclasses.replace(sc_full, heads=args.heads)
+    if args.scaling == "strong":
+        # this rank's heads of the one input (the same bytes the one-rank run draws for them)
+        h0, h1 = shard.head_range(rank, world, sc_full.heads)
+        q, k, v = shard.make_shard_inputs(sc_full, rank, world, device=dev)
+    else:
+        h0, h1 = 0, sc_full.heads
+        q, k, v = synth.make_qkv(sc_full.n_q, sc_full.n_kv, sc_full.heads, sc_full.head_dim,
+                                 rank_seeds(sc_full, rank), device=dev)
+    sc = dataclasses.replace(sc_full, heads=h1 - h0)   # what this rank computes
+    if sc.heads < 1:
+        raise SystemExit(f"rank {rank}: no heads to run ({sc_full.heads} heads over {world} ranks)")
     plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode)
     kmax = int(plan.k_total)
     ws = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
@@ -394,35 +451,65 @@ def run_ours(args, rank, world, local_rank):
     t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     status = S.device_status()
     ms, t_sel, t_att = max_over_ranks([ms, t_sel, t_att], dev, world)
+    flops_all = sum_over_ranks(flops, dev, world)
+    sel_bytes_all = sum_over_ranks(sel_bytes, dev, world)
 
     peaks, peak_src = load_peaks()
-    attn_tflops = flops / (t_att * 1e-3) / 1e12
-    sel_gbs = sel_bytes / (t_sel * 1e-3) / 1e9
-    peak_t = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    # Per GPU: this rank's share of the work over the slowest rank's kernel time.
+    attn_tflops = flops_all / world / (t_att * 1e-3) / 1e12
+    sel_gbs = sel_bytes_all / world / (t_sel * 1e-3) / 1e9
+    # The attention launch is a ~15 ms kernel timed on its own events, so its roofline is the
+    # burst cuBLAS figure; the sustained (power-capped, seconds-long) figure is reported beside it.
+    peak_t = float(peaks["bf16_tflops"])
+    peak_t_sus = float(peaks.get("bf16_tflops_sustained", peak_t))
     peak_hbm = float(peaks["hbm_gbs"])
+    read_gbs = read_bandwidth_probe(dev)
+    read_peak = max(peak_hbm, read_gbs)
+    traffic = recorded_traffic("attn_sparse_kernel<128>", sc_full.name if not args.heads else "")
+    if traffic is not None:
+        traffic *= sc.heads / sc_full.heads   # the record is per launch over all heads
     result = {
         "metric": METRIC,
-        "value": whole_job_tflops(flops, ms, world),
+        "value": whole_job_tflops(flops_all, ms),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(sc, args),
+        "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(sc_full, args, world),
         "gpu_launches": launches_per_step * args.steps,
         "attn": {"ms": t_att, "tflops": attn_tflops, "frac_of_peak": attn_tflops / peak_t,
-                 "frac_of_burst_peak": attn_tflops / float(peaks["bf16_tflops"]),
-                 "kept_tile_tflop": flops / 1e12, "kept_blocks_per_row": kmax},
+                 "frac_of_sustained_peak": attn_tflops / peak_t_sus,
+                 "kept_tile_tflop": flops_all / 1e12, "kept_blocks_per_row": kmax},
         "select": {"us": t_sel * 1e3, "gbs": sel_gbs, "frac_of_hbm": sel_gbs / peak_hbm,
-                   "bytes": sel_bytes, "share_of_step": t_sel / (t_sel + t_att)},
+                   "read_probe_gbs": read_gbs, "frac_of_read_peak": sel_gbs / read_peak,
+                   "frac_of_spec": sel_gbs / HBM_SPEC_GBS, "bytes": sel_bytes_all,
+                   "share_of_step": t_sel / (t_sel + t_att),
+                   "note": "frac_of_hbm divides by the measured copy rate (read + write); "
+                           "frac_of_read_peak by the higher of that and a read-only reduction probe "
+                           "timed in this run; frac_of_spec by the 7.7 TB/s HGX B200 figure"},
         "us_per_scale": ms * 1e3,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak_t,
-                     "traffic": recorded_traffic("attn_sparse_kernel<128>", sc.name if not args.heads else ""),
+                     "frac": attn_tflops / peak_t, "traffic": traffic,
                      "kernel": "attn_sparse_kernel<128>",
-                     "peak_source": f"{peak_src} bf16 sustained (kernel inside a back-to-back step loop)"},
+                     "peak_source": f"{peak_src} bf16 burst (the kernel is timed alone, one ~15 ms launch)",
+                     "sustained_peak": peak_t_sus, "frac_of_sustained": attn_tflops / peak_t_sus},
         "device_status": int(status),
     }
     clocks_summary = clocks.summary()
     result["clocks"] = clocks_summary
+    if world > 1 and args.gather_o:
+        # Optional: one all-gather of O across ranks (a caller whose next layer needs every
+        # head); not part of the step, which has no collective.
+        shard.gather_heads(o, rank, world, sc_full.heads)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        g0.record(stream)
+        full_o = shard.gather_heads(o, rank, world, sc_full.heads)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gms, = max_over_ranks([g0.elapsed_time(g1)], dev, world)
+        result["allgather_o"] = {"ms": gms, "bytes_per_rank_out": int(o.numel() * 2),
+                                 "gbs_per_rank": full_o.numel() * 2 * (world - 1) / world / (gms * 1e-3) / 1e9}
+        del full_o
 
     # The 64-token block variant on the same input (the pages' block-size ablation): same path,
     # block = 64 for the partition, the scores, the Top-K and the attention tiles.
@@ -506,7 +593,8 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_reuse and not args.heads and sc.clip >= 2 and sc.n_text % 128 == 0 and sc.n_ctx % 128 == 0:
         from block_sparse_attention_tok_b200 import reuse
         q_prev = synth.make_prev_clip_queries(sc.n_q, sc.heads, sc.head_dim,
-                                              [500000 + h + 1000 * rank for h in range(sc.heads)], device=dev)
+                                              [500000 + h0 + h + (1000 * rank if args.scaling == "weak" else 0)
+                                               for h in range(sc.heads)], device=dev)
         reuse.reference_reuse(q, q_prev, k, v, *seg, 0.15, workspace=ws)   # warm-up
         r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         r0.record(stream)
@@ -596,11 +684,11 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         ems, serial_ms = max_over_ranks([a.elapsed_time(b) / n_e2e, serial_ms], dev, world)
-        result["e2e"] = {"value": whole_job_tflops(flops, ems, world), "unit": "TFLOP/s",
+        result["e2e"] = {"value": whole_job_tflops(flops_all, ems), "unit": "TFLOP/s",
                          "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                          "d2h_bytes_per_step": int(ho.numel() * 2), "ms_per_step": ems, "steps": n_e2e,
                          "pipelined": f"{n_chunks} head chunks per step on three streams (H2D / forward / D2H)",
-                         "serial_value": whole_job_tflops(flops, serial_ms, world), "serial_ms_per_step": serial_ms}
+                         "serial_value": whole_job_tflops(flops_all, serial_ms), "serial_ms_per_step": serial_ms}
         del hq, hk, hv, ho, ws_c
 
     if world == 1 and not args.no_schedule and not args.heads:
@@ -622,8 +710,35 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _spawned_rank(local_rank: int, world: int, port: int, argv):
+    """Entry of a rank started by launch_ranks: the torchrun environment, then main()."""
+    os.environ.update(RANK=str(local_rank), LOCAL_RANK=str(local_rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.argv = [sys.argv[0]] + list(argv)
+    rc = main()
+    if rc:
+        raise SystemExit(rc)
+
+
+def launch_ranks(n: int) -> int:
+    """`--gpus N` without a torchrun environment: start N ranks (one process per GPU, spawned)."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_spawned_rank, args=(n, _free_port(), sys.argv[1:]), nprocs=n, join=True,
+                       start_method="spawn")
+    return 0
+
+
 def main():
     args = parse()
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(args.gpus)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

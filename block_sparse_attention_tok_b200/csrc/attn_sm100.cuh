@@ -189,7 +189,7 @@ __device__ __forceinline__ float row_max(const uint32_t (&r)[NC][32]) {
 
 // 2^x on the FMA pipe for a pair of arguments x <= 8: n = round(x) with the 1.5*2^23
 // shifter, f = x - n in [-1/2, 1/2], 2^f by a degree-3 polynomial (coefficients from
-// exp2_poly_fit.py: Chebyshev-node least squares of the relative error, max 1.2e-4), and
+// tests/exp2_poly_fit.py: Chebyshev-node least squares of the relative error, max 1.2e-4), and
 // 2^n added into the exponent field. Arguments below -125 are clamped there (2^-125 is
 // far below anything a bf16 P or the fp32 row sum can register).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {

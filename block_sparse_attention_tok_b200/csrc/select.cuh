@@ -13,9 +13,12 @@
 //                    stored as two bf16 numbers hi = bf16(m), lo = bf16(m - hi).
 //   score_tc_kernel  S = qbar kbar^T / sqrt(d) on the tensor cores: persistent CTAs over
 //                    128 x 128 tiles of (query block, KV block) pairs, TMA-fed,
-//                    tcgen05.mma accumulating hi.hi + hi.lo + lo.hi in fp32 tensor memory
-//                    (the dropped lo.lo term and the bf16 rounding of lo keep the error near
-//                    2^-16 sum_c |qbar_c kbar_c|/sqrt(d)).
+//                    tcgen05.mma accumulating hi.hi + hi.lo + lo.hi in fp32 tensor memory.
+//                    Error bound: hi = bf16(m), lo = bf16(m - hi) leave e = m - hi - lo with
+//                    |e| <= 2^-16 |m| and |lo| <= 2^-8 |m|, so each dropped term (hi_q e_k,
+//                    e_q k, lo_q lo_k) is at most about 2^-16 |q_c k_c|; with the fp32
+//                    accumulation of 3d products the error stays below
+//                    2^-14 sum_c |qbar_c kbar_c| / sqrt(d), far inside the 1e-3 tie gap.
 //   topk_warp_kernel one warp per (head, query block) row, staged in shared memory with
 //                    16-byte copies, each lane owning a contiguous run: the K-th largest key
 //                    is bracketed by a value histogram, then resolved among <= 32 keys

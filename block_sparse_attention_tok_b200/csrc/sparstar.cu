@@ -582,9 +582,15 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
                             int head_dim, int clip, double density, int budget_mode, int32_t* idx, int32_t* cnt,
                             int32_t kmax, void* stream) {
   // Sizes are checked before any CUDA call, so an oversized request never touches the device.
-  size_t need = 0;
-  int rc = sparstar_workspace_size(heads, n_q, seg, head_dim, &need);
+  sparstar_plan plan;
+  int rc = sparstar_make_plan(n_q, seg, clip, density, budget_mode, &plan);
   if (rc != SPARSTAR_OK) return rc;
+  size_t need = 0;
+  if ((rc = sparstar_workspace_size(heads, n_q, seg, head_dim, &need)) != SPARSTAR_OK) return rc;
+  // Rows that do not depend on the scores (forced-only, or every block kept) use no scratch.
+  if (!(plan.k_topk > 0 && plan.k_topk < plan.n_cand))
+    return sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
+                           nullptr, 0, stream);
   if (need > SPARSTAR_NOALLOC_SCRATCH_BYTES) return SPARSTAR_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sparstar::kMaxDevices) return SPARSTAR_ERR_CUDA;

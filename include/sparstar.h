@@ -159,8 +159,11 @@ int sparstar_forward(const void* q, const void* k, const void* v, int heads, int
  * all device memory through its own pool, a plugin that must not allocate, or code that
  * runs while a memory-capping policy is in force.
  * The array holds SPARSTAR_NOALLOC_SCRATCH_BYTES bytes on every device that loads the
- * library, until the process exits. Sizes whose sparstar_workspace_size() exceeds it are
- * rejected with SPARSTAR_ERR_UNSUPPORTED before anything is enqueued.
+ * library, until the process exits. When the rows depend on the scores (0 < k_topk < n_cand
+ * in the plan), sizes whose sparstar_workspace_size() exceeds it are rejected with
+ * SPARSTAR_ERR_UNSUPPORTED before anything is enqueued; rows that do not depend on the
+ * scores (forced-only rows, or rows keeping every block) use no scratch and have no limit
+ * beyond those of sparstar_select.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture.
  * All calls on a device share the one array and it keeps the last call's contents; every

@@ -10,12 +10,14 @@ English abstract "SparSTAR: Sparse Attention for SpaceTime AutoRegressive Video 
 (newx.sg), section Abstract:
   1. split Q and the mixed KV context (text ‖ reference context ‖ current tokens) into
      128-token blocks                                    (方法概览, bullet 块划分与聚合评分);
-  2. mean-pool each block                                 (same bullet: 对块内向量取均值);
+  2. mean-pool each block (the same bullet: a block is represented by the average of its
+     token vectors);
   3. score every (query block, key block) pair from the pooled vectors (same bullet);
   4. keep the clip-aware conditioning blocks dense: text always, and in Clip 1 also the
      image-pyramid blocks                                 (bullet clip感知保留策略);
   5. fill each query-block row with a joint Top-K over the remaining key blocks
-     (方法概览 first paragraph: 对其余块联合Top-K选择), separately for every head
+     (方法概览, first paragraph: one Top-K over all blocks not kept by rule), separately for
+     every head
      (bullet per-head动态掩码);
   6. run forward-only attention over the kept blocks only (bullet FastFlex执行路径).
 The pages print no formulas, code or worked example for SparSTAR. Readings of the open
@@ -43,7 +45,7 @@ from typing import Sequence, Tuple
 
 import numpy as np
 
-BLOCK = 128  # 方法概览: "按128-token块划分"
+BLOCK = 128  # block edge of the partition, in tokens (方法概览)
 
 BUDGET_LITERAL = 0      # rows hold max(ceil(density * nkb), n_forced) blocks
 BUDGET_CANDIDATES = 1   # Top-K keeps ceil(density * n_candidates) non-forced blocks
@@ -109,7 +111,8 @@ def row_budget(nkb: int, n_forced: int, density: float, mode: int = BUDGET_LITER
 # --------------------------------------------------------------------------- step 2
 
 def pool_blocks(x: np.ndarray, block: int = BLOCK) -> np.ndarray:
-    """Mean of the token vectors inside each block, [N, d] -> [nb, d] (方法概览: 对块内向量取均值).
+    """Mean of the token vectors inside each block, [N, d] -> [nb, d] (方法概览, bullet 块划分与聚合评分:
+    the block average).
 
     A ragged last block is averaged over its valid tokens only.
     """

@@ -21,3 +21,15 @@ def cuda_lib():
         pytest.skip("no CUDA device")
     from block_sparse_attention_tok_b200 import sparstar
     return sparstar.load()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print, per checked configuration, how many mask rows and output blocks were compared."""
+    try:
+        from tests.parity import LOG
+    except Exception:  # the parity module was never imported (CPU-only run)
+        return
+    if LOG:
+        terminalreporter.write_line("parity coverage (GPU vs oracle):")
+        for line in LOG:
+            terminalreporter.write_line("  " + line)

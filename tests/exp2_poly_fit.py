@@ -4,7 +4,7 @@ Method: Cody-Waite style range reduction 2^x = 2^n * 2^f with n = round(x), f in
 and 2^f approximated by a polynomial fitted by weighted least squares on Chebyshev nodes of
 [-1/2, 1/2] (a near-minimax fit of the relative error), evaluated with Horner's rule. The
 constant term is pinned to 1 so that 2^0 is exact. Run this file to print the coefficients
-that exp2_poly2() in attn_sm100.cuh uses and the fit's maximum relative error.
+that exp2_poly2() in the attention kernel (csrc/attn_sm100.cuh) uses and the fit's maximum relative error.
 """
 import numpy as np
 

@@ -24,7 +24,7 @@ def _kernel_coeffs():
 
 
 def _fit():
-    spec = importlib.util.spec_from_file_location("fit", os.path.join(CSRC, "exp2_poly_fit.py"))
+    spec = importlib.util.spec_from_file_location("fit", os.path.join(os.path.dirname(__file__), "exp2_poly_fit.py"))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod.fit(3)

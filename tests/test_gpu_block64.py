@@ -6,15 +6,13 @@ With 64-token blocks a query block is 64 rows of the kernel's 128-row MMA tile (
 last one alone, its second half masked), and rows with more than 3,965 candidates go
 through the radix Top-K.
 """
-import math
-
 import numpy as np
 import pytest
 import torch
 
 from block_sparse_attention_tok_b200 import synth
 from oracle import sparstar_oracle as O
-from tests.parity import bits, check_masks, check_output, LSE_ABS
+from tests.parity import bits, check_output, run_and_check, LSE_ABS
 
 pytestmark = pytest.mark.gpu
 B = 64
@@ -30,36 +28,12 @@ def _f64(x):
     return O.bf16_bits_to_f64(x)
 
 
-def _run(S, q, k, v, n_text, n_ctx, n_cur, clip, density, mode=0, qblocks=None, heads=None):
-    H, n_q, d = q.shape
-    heads = list(range(H)) if heads is None else heads
-    o, lse, idx, cnt = S.forward(q, k, v, n_text, n_ctx, n_cur, clip, density, mode, block=B)
-    _, _, scores = S.select(q, k, n_text, n_ctx, n_cur, clip, density, mode, want_scores=True, block=B)
-    assert S.device_status() == S.OK
-    plan = S.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode, block=B)
-    sel = torch.tensor(heads, device=q.device)
-    qb, kb, vb = bits(q[sel]), bits(k[sel]), bits(v[sel])
-    ref = [O.select_head(_f64(qb[i]), _f64(kb[i]), n_text, n_ctx, clip, density, mode, block=B)
-           for i in range(len(heads))]
-    ref_idx, ref_S = np.stack([r[0] for r in ref]), np.stack([r[1] for r in ref])
-    gidx, gcnt = idx[sel].cpu().numpy(), cnt[sel].cpu().numpy()
-    stats = check_masks(gidx, gcnt, ref_idx, ref_S, int(plan.n_forced), int(plan.k_topk))
-    got_S = scores[sel].cpu().numpy()
-    for hi in range(len(heads)):
-        qbar, kbar = O.pool_blocks(_f64(qb[hi]), B), O.pool_blocks(_f64(kb[hi]), B)
-        bound = 2.0 ** -14 * (np.abs(qbar) @ np.abs(kbar).T) / math.sqrt(d) + 1e-7
-        assert (np.abs(got_S[hi] - ref_S[hi]) <= bound).all()
-    o_np, lse_np = o[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
-    nqb = int(plan.nqb)
-    for hi in range(len(heads)):
-        qbl = range(nqb) if qblocks is None else qblocks(nqb)
-        qbl = [i for i in qbl if (gidx[hi, i, :ref_idx.shape[2]] == ref_idx[hi, i]).all()]
-        outs = O.block_sparse_attention(_f64(qb[hi]), _f64(kb[hi]), _f64(vb[hi]), ref_idx[hi], qbl, block=B)
-        for i, (o_ref, lse_ref) in zip(qbl, outs):
-            s, e = O.block_token_range(i, n_q, B)
-            check_output(o_np[hi, s:e], o_ref, f"h{heads[hi]} qb{i}")
-            assert np.abs(lse_np[hi, s:e] - lse_ref).max() <= LSE_ABS
-    return stats, plan
+def _run(S, q, k, v, n_text, n_ctx, n_cur, clip, density, mode=0, qblocks=None, out_heads=None, label=None):
+    """Masks of every head by the gap rule, scores within the split-precision bound, outputs of
+    `out_heads` on `qblocks` plus every block whose mask differs (oracle on the GPU's kept list)."""
+    stats = run_and_check(S, O, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, block=B, qblocks=qblocks,
+                          out_heads=out_heads, label=label)
+    return stats, S.make_plan(q.shape[1], n_text, n_ctx, n_cur, clip, density, mode, block=B)
 
 
 @pytest.mark.parametrize("d,n_q,n_text,n_ctx,n_cur,clip,density", [
@@ -135,14 +109,14 @@ def test_block64_pairs_odd_even_and_ragged(S, d, kk):
 
 @pytest.mark.slow
 def test_block64_final_scale_sampled(S):
-    """The 720p Clip-2 final scale with 64-token blocks (every mask row of 3 heads checked,
-    outputs on sampled query blocks)."""
+    """The 720p Clip-2 final scale with 64-token blocks: every mask row of all 32 heads, outputs
+    of three heads on sampled query blocks plus every block whose mask differs."""
     sc = synth.FINAL_CLIP2
     q, k, v = synth.make_scale_inputs(sc, device="cuda")
     rng = np.random.default_rng(64)
     stats, plan = _run(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density,
                        qblocks=lambda n: sorted({0, n - 1, *rng.choice(n, 3, replace=False).tolist()}),
-                       heads=[0, 15, 31])
-    print(stats)
+                       out_heads=[0, 15, 31], label=f"{sc.name} block 64")
+    assert stats["rows"] == sc.heads * int(plan.nqb)
     del q, k, v
     torch.cuda.empty_cache()

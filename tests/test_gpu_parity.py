@@ -5,15 +5,13 @@ bench.py launches them) are compared on every mask row and on sampled query bloc
 the attention output. Inputs are seeded (block_sparse_attention_tok_b200.synth); the
 oracle always reads the exact bytes the GPU used.
 """
-import math
-
 import numpy as np
 import pytest
 import torch
 
 from block_sparse_attention_tok_b200 import synth
 from oracle import sparstar_oracle as O
-from tests.parity import bits, check_masks, check_output, LSE_ABS
+from tests.parity import bits, check_output, run_and_check, LSE_ABS
 
 pytestmark = pytest.mark.gpu
 
@@ -27,43 +25,13 @@ def _oracle_attention(qb, kb, vb, rows, h, qblocks, d):
     return O.block_sparse_attention(qf, kf, vf, rows, qblocks)
 
 
-def _run_case(lib, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, qblocks_per_head=None, heads=None):
-    """Forward on the GPU; the mask rule on every row of the checked heads; outputs on the
-    query blocks (all, or qblocks_per_head(nqb)) whose mask equals the oracle's."""
-    S = lib
-    H, n_q, d = q.shape
-    heads = list(range(H)) if heads is None else list(heads)
-    o, lse, idx, cnt = S.forward(q, k, v, n_text, n_ctx, n_cur, clip, density, mode)
-    _, _, scores = S.select(q, k, n_text, n_ctx, n_cur, clip, density, mode, want_scores=True)
-    assert S.device_status() == S.OK
-    plan = S.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode)
-    sel = torch.tensor(heads, device=q.device)
-    qb, kb, vb = bits(q[sel]), bits(k[sel]), bits(v[sel])
-    ref = [O.select_head(_f64(qb[i]), _f64(kb[i]), n_text, n_ctx, clip, density, mode) for i in range(len(heads))]
-    ref_idx = np.stack([r[0] for r in ref])
-    ref_S = np.stack([r[1] for r in ref])
-    gidx, gcnt = idx[sel].cpu().numpy(), cnt[sel].cpu().numpy()
-    stats = check_masks(gidx, gcnt, ref_idx, ref_S, int(plan.n_forced), int(plan.k_topk))
-    # The kernel's scores (tensor cores, block means split into bf16 hi + lo, hi.hi + hi.lo +
-    # lo.hi in fp32) against the fp64 definition: each operand keeps ~16 bits, so the error
-    # is below 2^-14 * sum_c |qbar_c kbar_c| / sqrt(d), plus fp32 accumulation.
-    got_S = scores[sel].cpu().numpy()
-    for hi in range(len(heads)):
-        qbar = O.pool_blocks(_f64(qb[hi]))
-        kbar = O.pool_blocks(_f64(kb[hi]))
-        bound = 2.0 ** -14 * (np.abs(qbar) @ np.abs(kbar).T) / math.sqrt(d) + 1e-7
-        assert (np.abs(got_S[hi] - ref_S[hi]) <= bound).all(), "score error above the split-precision bound"
-    o_np, lse_np = o[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
-    nqb = int(plan.nqb)
-    for hi in range(len(heads)):
-        qbl = range(nqb) if qblocks_per_head is None else qblocks_per_head(nqb)
-        qbl = [i for i in qbl if (gidx[hi, i, :ref_idx.shape[2]] == ref_idx[hi, i]).all()]
-        outs = _oracle_attention(qb, kb, vb, ref_idx[hi], hi, qbl, d)
-        for i, (o_ref, lse_ref) in zip(qbl, outs):
-            s, e = O.block_token_range(i, n_q)
-            check_output(o_np[hi, s:e], o_ref, f"h{heads[hi]} qb{i}")
-            assert np.abs(lse_np[hi, s:e] - lse_ref).max() <= LSE_ABS
-    return stats
+def _run_case(lib, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, qblocks_per_head=None, out_heads=None,
+              label=None):
+    """Forward on the GPU; the mask rule on every row of every head; outputs on the query
+    blocks (all, or qblocks_per_head(nqb)) of `out_heads` (default all), plus every query
+    block whose mask differs from the oracle's, against the oracle on the GPU's kept list."""
+    return run_and_check(lib, O, q, k, v, n_text, n_ctx, n_cur, clip, density, mode, qblocks=qblocks_per_head,
+                         out_heads=out_heads, label=label)
 
 
 def _attn_with_oracle_mask(lib, q, k, v, rows_all, qblocks=None):
@@ -93,7 +61,7 @@ def S(cuda_lib):
 def test_tiny_clip2_scale_all_rows(S):
     sc = synth.TINY_CLIP2
     q, k, v = synth.make_scale_inputs(sc, device="cuda")
-    stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, 0)
+    stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, 0, label=sc.name)
     assert stats["identical"] == stats["rows"]
 
 
@@ -239,29 +207,45 @@ def _sampled(nqb):
     return sorted({0, nqb - 1, *rng.choice(nqb, 3, replace=False).tolist()})
 
 
+def _sampled3(nqb):
+    rng = np.random.default_rng(nqb + 1)
+    return sorted({0, nqb - 1, int(rng.integers(nqb))})
+
+
+# Heads whose outputs are compared at full size (masks and scores: every head).
+_OUT_HEADS = [0, 1, 7, 16, 23, 31]
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name", [synth.MID_CLIP1.name, synth.FINAL_CLIP1_RAGGED.name, synth.FINAL_CLIP2.name])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_full_size_scales(S, name, mode):
+    """The three large workloads, launched as bench.py launches them (all 32 heads in one call),
+    in both budget readings: every mask row of every head, every block score, and the outputs
+    of six heads on sampled query blocks plus every block whose mask differs from the oracle's."""
     sc = synth.WORKLOADS[name]
-    if mode == 1 and sc.clip == 2:
-        pytest.skip("the candidates budget differs from the literal one only where forced blocks fill the row")
     q, k, v = synth.make_scale_inputs(sc, device="cuda")
     stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode,
-                      qblocks_per_head=_sampled, heads=[0, 1, sc.heads // 2, sc.heads - 1])
-    print(name, mode, stats)
+                      qblocks_per_head=_sampled3, out_heads=_OUT_HEADS, label=f"{name} budget {mode}")
+    assert stats["rows"] == sc.heads * -(-sc.n_q // 128)
     del q, k, v
     torch.cuda.empty_cache()
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("scale_index", [0, 3])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("scale_index", [0, 1, 2, 3])
 @pytest.mark.parametrize("layer", [0, 35])
-def test_schedule_scales(S, scale_index, layer):
+def test_schedule_scales(S, scale_index, layer, mode):
+    """The four refined scales of the Clip-1 schedule at layers 0 and 35, both budget readings:
+    every mask row of all 32 heads; outputs of two heads on sampled query blocks plus every
+    block whose mask differs."""
     sc = synth.SCHEDULE_CLIP1[scale_index]
     q, k, v = synth.make_scale_inputs(sc, device="cuda", layer=layer, scale_index=scale_index)
-    _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, 0,
-              qblocks_per_head=_sampled, heads=[0, 31])
+    stats = _run_case(S, q, k, v, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, mode,
+                      qblocks_per_head=_sampled3, out_heads=[0, 31],
+                      label=f"schedule s{scale_index + 1} layer {layer} budget {mode}")
+    assert stats["rows"] == sc.heads * -(-sc.n_q // 128)
     del q, k, v
     torch.cuda.empty_cache()
 
@@ -308,3 +292,55 @@ def test_wider_index_buffer_and_single_head(S):
     (o_ref, lse_ref), = O.block_sparse_attention(qf, kf, vf, rows, [0])
     check_output(o.float().cpu().numpy()[0], o_ref, "single row")
     assert abs(float(lse.cpu()[0, 0]) - float(lse_ref[0])) <= LSE_ABS
+
+
+@pytest.mark.parametrize("n_q,segs,H,d,clip,density,mode", [
+    (1024, (256, 768, 1024), 2, 64, 2, 0.25, 0),      # the tiny Clip-2 scale
+    (300, (100, 300, 333), 3, 128, 2, 0.4, 0),        # ragged tails; nkb = 6 (not a multiple of 4)
+    (1, (128, 0, 129), 1, 64, 2, 0.5, 0),             # one query row, one ragged KV block
+    (640, (256, 512, 700), 2, 128, 1, 0.6, 1),        # Clip 1, candidates reading
+])
+def test_writes_stay_inside_outputs(S, n_q, segs, H, d, clip, density, mode):
+    """Every output of selection and attention sits inside a larger buffer whose guard bands
+    (before and after) hold a known pattern: after the calls the bands are unchanged, so no
+    kernel writes past its idx, cnt, score, workspace, o or lse range on these shapes."""
+    lib = S.load()
+    G = 4096                                  # guard elements on each side
+    n_kv = sum(segs)
+    q, k, v = synth.make_qkv(n_q, n_kv, H, d, [900 + h for h in range(H)], device="cuda")
+    plan = S.make_plan(n_q, *segs, clip, density, mode)
+    nqb, nkb, kt = int(plan.nqb), int(plan.nkb), int(plan.k_total)
+    kmax = kt + 3
+    idx_buf = torch.full((2 * G + H * nqb * kmax,), -77, dtype=torch.int32, device="cuda")
+    cnt_buf = torch.full((2 * G + H * nqb,), -77, dtype=torch.int32, device="cuda")
+    sc_buf = torch.full((2 * G + H * nqb * nkb,), -7.5, dtype=torch.float32, device="cuda")
+    ws_bytes = S.workspace_size(H, n_q, *segs, d)
+    ws_buf = torch.full((2 * G * 4 + ws_bytes,), 0xA5, dtype=torch.uint8, device="cuda")
+    o_buf = torch.full((2 * G + H * n_q * d,), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse_buf = torch.full((2 * G + H * n_q,), 3.0, dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream or None
+    for scores in (False, True):
+        rc = lib.sparstar_select(q.data_ptr(), k.data_ptr(), H, n_q, S.Segments(*segs), d, clip, density, mode,
+                                 idx_buf[G:].data_ptr(), cnt_buf[G:].data_ptr(), kmax,
+                                 sc_buf[G:].data_ptr() if scores else None, ws_buf[4 * G:].data_ptr(), ws_bytes, st)
+        assert rc == S.OK
+    rc = lib.sparstar_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), H, n_q, n_kv, d, idx_buf[G:].data_ptr(),
+                           cnt_buf[G:].data_ptr(), kmax, 0.0, o_buf[G:].data_ptr(), lse_buf[G:].data_ptr(), st)
+    assert rc == S.OK
+    assert S.device_status() == S.OK
+
+    def guards_intact(buf, n, fill, unit=1):
+        b = buf.cpu()
+        head, tail = b[:unit * G], b[unit * G + n:]
+        return bool((head == fill).all()) and bool((tail == fill).all())
+
+    assert guards_intact(idx_buf, H * nqb * kmax, -77)
+    assert guards_intact(cnt_buf, H * nqb, -77)
+    assert guards_intact(sc_buf, H * nqb * nkb, -7.5)
+    assert guards_intact(ws_buf, ws_bytes, 0xA5, unit=4)
+    assert guards_intact(o_buf, H * n_q * d, 3.0)
+    assert guards_intact(lse_buf, H * n_q, 3.0)
+    # inside idx, entries past K_total of each row keep the caller's values
+    rows = idx_buf[G:G + H * nqb * kmax].view(H, nqb, kmax).cpu()
+    assert bool((rows[:, :, kt:] == -77).all())
+    assert bool((cnt_buf[G:G + H * nqb].cpu() == kt).all())

@@ -34,6 +34,30 @@ def test_oversized_request_is_rejected_before_touching_the_device():
     assert rc == sparstar.ERR_UNSUPPORTED
 
 
+@pytest.mark.gpu
+def test_rows_without_scores_need_no_scratch():
+    """Forced-only rows (the Clip-1 720p scale read literally: K_topk = 0) do not depend on the
+    scores, so they take no scratch: a head count whose scratch would exceed the fixed array is
+    accepted and gives the regular selection's rows (q and k are not read for such rows)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = _lib()
+    H, n_q, segs, d = 256, 72000, (512, 8192, 72000), 128
+    plan = sparstar.make_plan(n_q, *segs, 1, 0.09375, 0)
+    assert int(plan.k_topk) == 0
+    assert sparstar.workspace_size(H, n_q, *segs, d) > sparstar.NOALLOC_SCRATCH_BYTES
+    dummy = torch.zeros(64, dtype=torch.bfloat16, device="cuda")    # never read for these rows
+    idx = torch.full((H, int(plan.nqb), int(plan.k_total)), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((H, int(plan.nqb)), -1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream or None
+    rc = lib.sparstar_select_noalloc(dummy.data_ptr(), dummy.data_ptr(), H, n_q, sparstar.Segments(*segs), d, 1,
+                                     0.09375, 0, idx.data_ptr(), cnt.data_ptr(), idx.shape[-1], stream)
+    assert rc == sparstar.OK
+    assert sparstar.device_status() == sparstar.OK
+    want = torch.arange(int(plan.k_total), dtype=torch.int32, device="cuda").expand_as(idx)
+    assert torch.equal(idx, want) and bool((cnt == int(plan.k_total)).all())
+
+
 def _call_noalloc(lib, q, k, segs, clip, density, mode, idx, cnt):
     H, n_q, d = q.shape
     stream = torch.cuda.current_stream().cuda_stream or None
