@@ -208,21 +208,22 @@ def whole_job_tflops(flops_all_ranks: float, ms_max: float) -> float:
     return flops_all_ranks / (ms_max * 1e-3) / 1e12
 
 
-def read_bandwidth_probe(dev, nbytes: int = 4 << 30, reps: int = 5) -> float:
-    """Best read-only streaming rate (GB/s) of a plain reduction over a buffer far larger than L2
-    (torch.sum of fp32 zeros, CUDA events): the denominator for read-only kernels such as the
-    selection, whose traffic is almost all reads, next to the copy figure (read + write)."""
+def read_bandwidth_probe(S, dev, nbytes: int = 4 << 30, reps: int = 5) -> float:
+    """Best read-only streaming rate (GB/s) over a buffer far larger than L2: the library's read
+    probe (the pooling kernel's 16-byte streaming loads, nothing written), CUDA events. The
+    denominator for the selection, whose traffic is almost all reads, next to the copy figure
+    (read + write)."""
     x = torch.zeros(nbytes // 4, dtype=torch.float32, device=dev)
-    torch.sum(x)
+    sink = S.read_probe(x)
     best = 0.0
     for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        torch.sum(x)
+        S.read_probe(x, sink)
         b.record()
         torch.cuda.synchronize()
         best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
-    del x
+    del x, sink
     torch.cuda.empty_cache()
     return best
 
@@ -463,7 +464,7 @@ def run_ours(args, rank, world, local_rank):
     peak_t = float(peaks["bf16_tflops"])
     peak_t_sus = float(peaks.get("bf16_tflops_sustained", peak_t))
     peak_hbm = float(peaks["hbm_gbs"])
-    read_gbs = read_bandwidth_probe(dev)
+    read_gbs = read_bandwidth_probe(S, dev)
     read_peak = max(peak_hbm, read_gbs)
     traffic = recorded_traffic("attn_sparse_kernel<128>", sc_full.name if not args.heads else "")
     if traffic is not None:
@@ -484,8 +485,8 @@ def run_ours(args, rank, world, local_rank):
                    "frac_of_spec": sel_gbs / HBM_SPEC_GBS, "bytes": sel_bytes_all,
                    "share_of_step": t_sel / (t_sel + t_att),
                    "note": "frac_of_hbm divides by the measured copy rate (read + write); "
-                           "frac_of_read_peak by the higher of that and a read-only reduction probe "
-                           "timed in this run; frac_of_spec by the 7.7 TB/s HGX B200 figure"},
+                           "frac_of_read_peak by the higher of that and the library's read-only streaming "
+                           "probe timed in this run; frac_of_spec by the 7.7 TB/s HGX B200 figure"},
         "us_per_scale": ms * 1e3,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_t, "traffic": traffic,

@@ -130,6 +130,30 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
+// Measurement aid: one read of n16 16-byte chunks with the pooling kernel's streaming loads
+// (grid-stride, four loads in flight per thread), XOR-folded so the loads are not dead code,
+// one atomicXor per warp into *sink. Its rate is the read-only streaming bandwidth.
+__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ src, int64_t n16,
+                                                         unsigned* __restrict__ sink) {
+  uint32_t acc = 0u;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ld_stream_16(src + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = ld_stream_16(src + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc ^= __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+  if ((threadIdx.x & 31) == 0) atomicXor(sink, acc);
+}
+
 // ------------------------------------------------------------------------ scores
 
 template <int D>

@@ -608,6 +608,19 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
                          scratch, SPARSTAR_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+int sparstar_read_probe(const void* src, size_t bytes, unsigned* sink, void* stream) {
+  if (bytes == 0) return SPARSTAR_OK;
+  if (src == nullptr || sink == nullptr || !aligned16(src) || (bytes & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(sink) & 3u) != 0)
+    return SPARSTAR_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  read_probe_kernel<<<static_cast<unsigned>(dev->sms) * 4u, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<int64_t>(bytes / 16), sink);
+  return launch_status();
+}
+
 int sparstar_selftest_wait_timeout(void* stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);

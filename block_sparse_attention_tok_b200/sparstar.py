@@ -86,6 +86,7 @@ _SIGNATURES.update({
                                         _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "sparstar_topk": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _c.c_void_p, _c.c_void_p,
                                  _c.c_int32, _c.c_void_p]),
+    "sparstar_read_probe": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_void_p, _c.c_void_p]),
 })
 NOALLOC_SCRATCH_BYTES = 128 << 20
 
@@ -315,6 +316,18 @@ def select_noalloc(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_
                                           float(density), int(budget_mode), _ptr(idx), _ptr(cnt), idx.shape[-1],
                                           _stream_ptr(stream)), "sparstar_select_noalloc")
     return idx, cnt
+
+
+def read_probe(buf: torch.Tensor, sink: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Measurement aid: one streaming read of `buf` (a contiguous CUDA tensor whose size is a
+    multiple of 16 bytes), XOR-folded into a 4-byte sink, which is returned."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    _check(load().sparstar_read_probe(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), _stream_ptr(stream)),
+           "sparstar_read_probe")
+    return sink
 
 
 def device_status(clear: bool = True, stream=None) -> int:

@@ -246,6 +246,13 @@ int sparstar_device_status(void* stream, int clear);
  * and the CUDA context stays usable. Requires an sm_100 device. */
 int sparstar_selftest_wait_timeout(void* stream);
 
+/* Measurement aid, not a step of the method: reads `bytes` bytes at `src` (device, 16-byte
+ * aligned, a multiple of 16) once, with the streaming 16-byte loads of the pooling kernel,
+ * and XORs them into *sink (device, 4 bytes). Its duration gives the read-only streaming
+ * bandwidth that the read-bound selection is measured against (a copy reads and writes).
+ * bytes == 0 is a no-op; bad pointers or sizes give SPARSTAR_ERR_ARG. */
+int sparstar_read_probe(const void* src, size_t bytes, unsigned* sink, void* stream);
+
 /* Static text for a return code (never NULL). */
 const char* sparstar_strerror(int code);
 

@@ -353,12 +353,61 @@ def reference_reuse_report(q_now: np.ndarray, q_prev: np.ndarray, k: np.ndarray,
     e_reused = reference_mass(q_now, k, reused, n_text, n_ctx, qblocks, sm_scale, block)
     return fresh, reused, e_fresh, e_reused
 
+# --------------------------------------------------------------------------- mask reuse across scales
+
+def raster_block_map(grid_now: Sequence[int], grid_prev: Sequence[int], block: int = BLOCK) -> np.ndarray:
+    """For every block of a scale's current tokens, laid out on grid_now = (T', H', W') in raster
+    order (frame, row, column), the block of the previous scale's grid_prev = (T, H, W) that holds
+    the nearest raster position (digest section 关键结果与论文证据, bullet 重算频率, Figure 5:
+    a mask computed at one scale and reused at the next needs this correspondence; the pages do
+    not give it). A block is represented by its middle token c = start + (n - 1) // 2; along
+    each axis the new cell centre (x + 1/2) / X' falls in the old cell floor((2x + 1) X / (2 X')),
+    clipped to the last cell; the old token is unravelled back to a raster index and divided
+    by the block size."""
+    Tn, Hn, Wn = (int(x) for x in grid_now)
+    To, Ho, Wo = (int(x) for x in grid_prev)
+    n_now = Tn * Hn * Wn
+    out = np.empty(num_blocks(n_now, block), dtype=np.int64)
+    for b in range(len(out)):
+        s, e = block_token_range(b, n_now, block)
+        c = s + (e - s - 1) // 2
+        t, rem = divmod(c, Hn * Wn)
+        h, w = divmod(rem, Wn)
+        to = min(To - 1, (2 * t + 1) * To // (2 * Tn))
+        ho = min(Ho - 1, (2 * h + 1) * Ho // (2 * Hn))
+        wo = min(Wo - 1, (2 * w + 1) * Wo // (2 * Wn))
+        out[b] = ((to * Ho + ho) * Wo + wo) // block
+    return out
+
+
+def map_scores(S_prev: np.ndarray, n_prefix_blocks: int, grid_prev: Sequence[int], grid_now: Sequence[int],
+               block: int = BLOCK) -> np.ndarray:
+    """Block scores of the previous scale carried to the current one (reuse instead of
+    recompute, Figure 5): S_now[i', j'] = S_prev[m(i'), c(j')], m = raster_block_map (query
+    blocks are current-scale blocks), c(j') = j' for the KV prefix of text and reference-context
+    blocks (the same tokens at every scale of a clip) and n_prefix + m(j' - n_prefix) for the
+    current-scale blocks. S_prev is [nqb_prev, n_prefix + nb_cur_prev]."""
+    m = raster_block_map(grid_now, grid_prev, block)
+    cols = np.concatenate([np.arange(n_prefix_blocks), n_prefix_blocks + m])
+    assert S_prev.shape == (num_blocks(int(np.prod(grid_prev)), block),
+                            n_prefix_blocks + num_blocks(int(np.prod(grid_prev)), block))
+    return S_prev[np.ix_(m, cols)]
+
+
+def reused_rows(S_prev: np.ndarray, n_prefix_blocks: int, grid_prev: Sequence[int], grid_now: Sequence[int],
+                n_forced: int, k_topk: int, block: int = BLOCK) -> np.ndarray:
+    """Kept blocks of the current scale chosen from the previous scale's mapped scores: the
+    clip-aware forced prefix, then the current scale's own budget of K_topk by the joint Top-K
+    rule (ties to the lower index), exactly as a fresh selection but without new scores."""
+    return select_rows(map_scores(S_prev, n_prefix_blocks, grid_prev, grid_now, block), n_forced, k_topk)
+
+
 __all__ = [
     "BLOCK", "BUDGET_LITERAL", "BUDGET_CANDIDATES", "bf16_bits_to_f64", "num_blocks",
     "block_token_range", "forced_block_count", "row_budget", "pool_blocks", "block_scores",
     "select_rows", "select_row", "select_head", "select", "kept_token_index", "attend_rows",
     "block_sparse_attention", "dense_attention", "retained_mass", "block_energy",
     "kept_token_count", "dense_probabilities", "token_topk_bound", "mass_report", "reference_mass",
-    "reference_reuse_report",
+    "reference_reuse_report", "raster_block_map", "map_scores", "reused_rows",
 ]
 

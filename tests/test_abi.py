@@ -165,3 +165,11 @@ def test_topk_null_and_misaligned_pointers(lib):
     assert lib.sparstar_topk(0x1002, 4, 10, 2, 3, 0x2000, 0x3000, 8, None) == sparstar.ERR_ARG    # not 4-byte aligned
     assert lib.sparstar_topk(0x1000, 4, 10, 2, 3, None, 0x3000, 8, None) == sparstar.ERR_ARG
     assert lib.sparstar_topk(0x1000, 0, 10, 2, 3, None, None, 8, None) == sparstar.OK             # rows == 0: no-op
+
+
+def test_read_probe_rejects_bad_arguments_before_launch(lib):
+    assert lib.sparstar_read_probe(None, 64, 0x2000, None) == sparstar.ERR_ARG         # no source
+    assert lib.sparstar_read_probe(0x1008, 64, 0x2000, None) == sparstar.ERR_ARG       # not 16-byte aligned
+    assert lib.sparstar_read_probe(0x1000, 40, 0x2000, None) == sparstar.ERR_ARG       # not a multiple of 16
+    assert lib.sparstar_read_probe(0x1000, 64, None, None) == sparstar.ERR_ARG         # no sink
+    assert lib.sparstar_read_probe(0x1000, 0, None, None) == sparstar.OK               # empty: no-op

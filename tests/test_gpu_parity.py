@@ -344,3 +344,15 @@ def test_writes_stay_inside_outputs(S, n_q, segs, H, d, clip, density, mode):
     rows = idx_buf[G:G + H * nqb * kmax].view(H, nqb, kmax).cpu()
     assert bool((rows[:, :, kt:] == -77).all())
     assert bool((cnt_buf[G:G + H * nqb].cpu() == kt).all())
+
+
+@pytest.mark.parametrize("n_words", [4, 4 * 1000003, 4 * (148 * 4 * 512 * 4 + 3)])
+def test_read_probe_reads_every_chunk_once(S, n_words):
+    """The bandwidth probe's XOR fold equals the XOR of every 32-bit word of the buffer (each
+    16-byte chunk read exactly once, including a tail that is not a multiple of the grid)."""
+    g = torch.Generator(device="cuda").manual_seed(n_words)
+    buf = torch.randint(-2**31, 2**31 - 1, (n_words,), dtype=torch.int32, device="cuda", generator=g)
+    sink = S.read_probe(buf)
+    assert S.device_status() == S.OK
+    want = np.bitwise_xor.reduce(buf.cpu().numpy().view(np.uint32))
+    assert int(sink.cpu().numpy().view(np.uint32)[0]) == int(want)

@@ -464,3 +464,75 @@ def test_reference_reuse_rows_follow_global_block_scores_and_grow_with_budget():
     assert fresh.min() >= 1 and fresh.max() <= 4 and reused.min() >= 1 and reused.max() <= 4
     _, _, ef_small, _ = O.reference_reuse_report(q_now, q_prev, k, 128, 512, 0.25, [0, 1, 2])
     assert np.all(ef >= ef_small)   # nested Top-K sets keep at least as much mass
+
+
+# ------------------------------------------------------------------ mask reuse across scales
+
+def _brute_block_map(grid_now, grid_prev, block):
+    """The old block under each new block's middle token, found by scanning every old cell per
+    axis with exact fractions (the old cell whose span [i/X, (i+1)/X) holds the new cell centre)."""
+    from fractions import Fraction
+    Tn, Hn, Wn = grid_now
+    To, Ho, Wo = grid_prev
+    n_now = Tn * Hn * Wn
+    out = []
+    for b in range(-(-n_now // block)):
+        s, e = b * block, min((b + 1) * block, n_now)
+        c = s + (e - s - 1) // 2
+        t, h, w = c // (Hn * Wn), (c // Wn) % Hn, c % Wn
+        cell = []
+        for x, X_new, X_old in ((t, Tn, To), (h, Hn, Ho), (w, Wn, Wo)):
+            centre = Fraction(2 * x + 1, 2 * X_new)
+            hits = [i for i in range(X_old) if Fraction(i, X_old) <= centre < Fraction(i + 1, X_old)]
+            assert len(hits) == 1
+            cell.append(hits[0])
+        out.append(((cell[0] * Ho + cell[1]) * Wo + cell[2]) // block)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("grid_now,grid_prev,block", [
+    ((8, 94, 96), (8, 64, 72), 128),     # the synthetic schedule's last two scales
+    ((8, 64, 72), (8, 32, 32), 128),
+    ((3, 7, 11), (5, 4, 9), 16),         # shrinking frames, odd sizes, ragged last blocks
+    ((2, 9, 13), (2, 9, 13), 64),        # same grid
+    ((1, 5, 7), (4, 6, 6), 8),
+])
+def test_raster_block_map_against_exact_cell_scan(grid_now, grid_prev, block):
+    assert np.array_equal(O.raster_block_map(grid_now, grid_prev, block), _brute_block_map(grid_now, grid_prev, block))
+
+
+def test_raster_block_map_closed_forms():
+    # same grid: identity
+    assert np.array_equal(O.raster_block_map((8, 64, 72), (8, 64, 72)), np.arange(288))
+    # 2x in height and width with one old row per block: new block b (half a new row) lies in old row b // 4
+    assert np.array_equal(O.raster_block_map((1, 8, 256), (1, 4, 128)), np.arange(16) // 4)
+    # 2x in frames with one frame per block: new frame b lies in old frame b // 2
+    assert np.array_equal(O.raster_block_map((4, 1, 128), (2, 1, 128)), np.arange(4) // 2)
+
+
+def test_map_scores_gathers_rows_and_columns():
+    grid_prev, grid_now, pre = (2, 8, 24), (2, 12, 32), 5          # 384 -> 768 tokens: 3 -> 6 blocks
+    nb_prev = 3
+    S_prev = 1000.0 * np.arange(nb_prev)[:, None] + np.arange(pre + nb_prev)[None, :]   # encodes (i, j)
+    S_now = O.map_scores(S_prev, pre, grid_prev, grid_now)
+    m = _brute_block_map(grid_now, grid_prev, 128)
+    assert S_now.shape == (6, pre + 6)
+    rows, cols = np.divmod(S_now, 1000.0)
+    assert np.array_equal(rows, np.repeat(m[:, None], pre + 6, axis=1))
+    assert np.array_equal(cols[:, :pre], np.tile(np.arange(pre), (6, 1)))            # prefix: same blocks
+    assert np.array_equal(cols[:, pre:], np.tile(pre + m, (6, 1)))                    # current: mapped blocks
+
+
+def test_reused_rows_keep_the_current_budget_and_equal_fresh_rows_on_the_same_grid():
+    rng = np.random.default_rng(11)
+    S_prev = rng.standard_normal((6, 4 + 6))
+    same = O.reused_rows(S_prev, 4, (1, 6, 128), (1, 6, 128), 1, 3)
+    assert np.array_equal(same, O.select_rows(S_prev, 1, 3))
+    grown = O.reused_rows(S_prev, 4, (1, 6, 128), (1, 12, 128), 1, 5)
+    assert grown.shape == (12, 6) and (np.diff(grown, axis=1) > 0).all() and (grown[:, 0] == 0).all()
+    # rows of new blocks that map to the same old block are identical
+    m = O.raster_block_map((1, 12, 128), (1, 6, 128))
+    for a in range(12):
+        for b in range(12):
+            if m[a] == m[b]:
+                assert np.array_equal(grown[a], grown[b])
