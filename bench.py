@@ -380,6 +380,51 @@ def run_schedule(S, dev, stream, layers: int = 36):
     return out
 
 
+def run_cross_scale(S, dev, stream):
+    """Mask reuse across scales (recompute frequency): the four sparsified scales of the Clip-1
+    schedule (layer 0, 32 heads, candidates reading: under the literal reading scales 2-4 keep
+    only the forced prefix, so every policy gives the same masks), under three policies:
+    recompute at every scale, every second scale, or once at the first scale. Per policy and
+    scale: the mean retained dense softmax mass of the mask and the selection time (fresh
+    selection, or score map + Top-K)."""
+    from block_sparse_attention_tok_b200 import reuse
+    mode = S.BUDGET_CANDIDATES
+    scales, lse_dense = [], []
+    for si, sc in enumerate(synth.SCHEDULE_CLIP1):
+        q, k, v = synth.make_scale_inputs(sc, device=dev, layer=0, scale_index=si)
+        scales.append(dict(q=q, k=k, v=v, seg=(sc.n_text, sc.n_ctx, sc.n_cur), grid=sc.grid, clip=sc.clip,
+                           density=sc.density))
+        nqb, nkb = -(-sc.n_q // 128), -(-sc.n_kv // 128)
+        all_idx = torch.arange(nkb, dtype=torch.int32, device=dev).expand(sc.heads, nqb, nkb).contiguous()
+        all_cnt = torch.full((sc.heads, nqb), nkb, dtype=torch.int32, device=dev)
+        _, lse = S.attn(q, k, v, all_idx, all_cnt)
+        lse_dense.append(lse)
+        del all_idx, all_cnt
+    out = {"workload": "Clip-1 schedule, layer 0, 32 heads; grids (frames, height, width) " +
+                       ", ".join(str(sc.grid) for sc in synth.SCHEDULE_CLIP1),
+           "budget": "candidates", "policies": {}}
+    reuse.cross_scale_masks(scales, "every_2", mode)   # warm-up
+    for policy in reuse.POLICIES:
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        masks = reuse.cross_scale_masks(scales, policy, mode)
+        b.record(stream)
+        torch.cuda.synchronize()
+        rows = []
+        for sc, (idx, cnt), ld in zip(scales, masks, lse_dense):
+            _, lse_kept = S.attn(sc["q"], sc["k"], sc["v"], idx, cnt)
+            _, e = S.retained_mass(lse_kept, ld, want_tokens=False)
+            rows.append(float(e.mean()))
+        out["policies"][policy] = {"retained_mean_per_scale": rows, "selection_ms_all_scales": a.elapsed_time(b)}
+        del masks
+    del scales, lse_dense
+    torch.cuda.empty_cache()
+    out["note"] = ("synthetic inputs are independent across scales, so reused masks act as uninformed ones; "
+                   "the pages' Figure 5 differences (1.73 / 0.79 dB) come from model activations")
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     from block_sparse_attention_tok_b200 import sparstar as S
     import torch.distributed as dist
@@ -696,6 +741,7 @@ def run_ours(args, rank, world, local_rank):
         del o, lse
         torch.cuda.empty_cache()
         result["schedule"] = run_schedule(S, dev, stream)
+        result["cross_scale"] = run_cross_scale(S, dev, stream)
 
     if rank == 0 and not args.no_cpu_baseline:
         n_h = min(4, q.shape[0])

@@ -16,14 +16,15 @@
 // mass_kernel computes R and its block means from the two LSEs. The bound needs the dense
 // logits again: bound_pass_kernel recomputes S = Q K^T for every (query block, key block)
 // tile on the tensor cores (TMA -> tcgen05.mma -> tensor memory) and bins x = log2 P_tu of
-// each row into 32 equal bins of a per-row interval. After a pass the row keeps the bin
-// holding its B-th largest value as the next interval and adds the count and mass of the
-// bins above it to its running totals; four passes narrow the interval from 64 to
-// 64/32^4 = 2^-14 (log2 units), and the last pass takes the boundary bin's mean for the
-// still missing values (relative error below 2^-15 * ln 2 of U). Bins are cells of one
-// fixed grid: y = log2 P + 64 is rounded once, and the bin of pass p is floor(y * 2^(5p-1))
-// (an exact power-of-two scaling), so a value's cell in pass p+1 always lies inside its cell
-// of pass p and no value is counted twice or lost at a bin edge.
+// each row into 32 equal bins of a per-row interval. The first three passes only count: after
+// each, the row keeps the bin holding its B-th largest value as the next interval and takes
+// the count of the bins above it off B. The last pass sums P over every value above the final
+// interval (width 64/32^4 = 2^-14 in log2 units) in registers, bins the few values inside it
+// by count and mass, and takes the boundary bin's mean for the still missing values
+// (relative error below 2^-15 * ln 2 of U). Bins are cells of one fixed grid:
+// y = log2 P + 64 is rounded the same way in every pass, and the bin of pass p is
+// floor(y * 2^(5p-1)) (an exact power-of-two scaling), so a value's cell in pass p+1 always
+// lies inside its cell of pass p and no value is counted twice or lost at a bin edge.
 #pragma once
 
 #include <cstdint>
@@ -37,6 +38,18 @@ namespace sparstar {
 constexpr int kBoundBins = 32;
 constexpr int kBoundPasses = 4;
 constexpr float kBoundLo = -64.0f;  // log2 P below 2^-64 never matters for a bound on mass
+constexpr float kBoundYTop = 63.999996185302734f;  // the largest float below 64 (= -kBoundLo)
+constexpr uint32_t kBoundMagicBits = 0x4B400000u;   // bit pattern of 1.5 * 2^23
+// Count histograms per thread in the counting passes: value e of a group of 8 updates histogram
+// e % kBoundSubs, so four read-modify-writes are independent (no shared-memory address can
+// repeat among them). Counts are 16-bit: a histogram gets 16 values a tile, so up to
+// kBoundMaxKvBlocks tiles never overflow one.
+constexpr int kBoundSubs = 4;
+constexpr int kBoundMaxKvBlocks = 65535 / 16;
+constexpr uint32_t kBoundCells = kBoundBins + 2;  // the interval's bins and two cells outside it
+// Last pass, inside a warp's region: a 32-bit count histogram [bin][lane] at 0 and the fp32
+// mass histogram [bin][lane] from here.
+constexpr uint32_t kBoundMassOffset = kBoundBins * 32 * 4;
 
 // 1 / bin width of a pass: widths 2, 1/16, 1/512, 1/16384 (pass 0 covers [-64, 0) in 32 bins)
 __device__ __forceinline__ float bound_inv_width(int pass) {
@@ -117,12 +130,16 @@ struct BoundConfig {
   static constexpr int kChunks = D / 64;
   static constexpr uint32_t kChunkBytes = 128 * 128;
   static constexpr uint32_t kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kThreads = 320;  // 8 binning warps + TMA warp + MMA warp
   static constexpr int kLoadWarp = 8;
   static constexpr int kMmaWarp = 9;
   static constexpr uint32_t kTmemCols = 256;  // S0, S1
-  static constexpr uint32_t kHistBytes = 8 * kBoundBins * 32 * 8;  // [warp][bin][lane] count + mass
+  // Per binning warp: kBoundSubs 16-bit count histograms [sub][bin + junk][lane] (the last pass
+  // reuses the region for one count histogram and a fp32 mass histogram); then 128 floats for
+  // the second half's row sums.
+  static constexpr uint32_t kWarpHistBytes = kBoundSubs * kBoundCells * 32 * 2;
+  static constexpr uint32_t kHistBytes = 8 * kWarpHistBytes + 128 * 4;
   static constexpr uint32_t kSmemBytes = 1024 + kTileBytes + kStages * kTileBytes + kHistBytes + 256;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
 };
@@ -147,9 +164,9 @@ __global__ void __launch_bounds__(BoundConfig<D>::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* q_tile = smem;
   uint8_t* ring = smem + C::kTileBytes;
-  uint32_t* hist_n = reinterpret_cast<uint32_t*>(ring + C::kStages * C::kTileBytes);  // [8][bins][32]
-  float* hist_m = reinterpret_cast<float*>(hist_n + 8 * kBoundBins * 32);            // [8][bins][32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(hist_m + 8 * kBoundBins * 32);
+  uint8_t* hist = ring + C::kStages * C::kTileBytes;                                 // [8][kWarpHistBytes]
+  float* above_part = reinterpret_cast<float*>(hist + 8 * C::kWarpHistBytes);        // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(above_part + 128);
   uint64_t* full = bars;                // [kStages]
   uint64_t* empty = full + C::kStages;  // [kStages]
   uint64_t* q_full = empty + C::kStages;
@@ -280,15 +297,24 @@ __global__ void __launch_bounds__(BoundConfig<D>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ binning warps
     // Warps w and w+4 share TMEM lane quarter w%4 (32 query rows); warp w bins key columns
-    // 0-63 of each S tile, warp w+4 columns 64-127, each into its own histogram.
+    // 0-63 of each S tile, warp w+4 columns 64-127, each into its own histograms.
+    //   passes 0 .. kBoundPasses-2: counts only, in 34 cells: cells 1..32 are the interval's
+    //     bins, cell 0 holds values one bin below it and cell 33 every other value outside it;
+    //   last pass: every value above the interval adds its P to a register sum, values inside
+    //     the interval go to count + mass bins (a handful per row), the rest is skipped.
     const int wq = warp & 3, half = warp >> 2;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    uint32_t* hn = hist_n + warp * kBoundBins * 32 + lane;  // stride 32 per bin: conflict-free
-    float* hm = hist_m + warp * kBoundBins * 32 + lane;
+    uint8_t* my_hist = hist + warp * C::kWarpHistBytes + lane * 2;    // [sub][cell][lane] u16
+    uint32_t* hn32 = reinterpret_cast<uint32_t*>(hist + warp * C::kWarpHistBytes) + lane;  // last pass
+    float* hm = reinterpret_cast<float*>(hist + warp * C::kWarpHistBytes + kBoundMassOffset) + lane;
+    static_assert(kBoundMassOffset + kBoundBins * 32 * 4 <= C::kWarpHistBytes, "last-pass histograms overflow");
+    constexpr uint32_t kCellBytes = 32 * 2;                              // one cell of all 32 lanes
+    constexpr uint32_t kSubBytes = kBoundCells * kCellBytes;
     const float inv_w = bound_inv_width(p.pass);
-    const bool first_pass = p.pass == 0;
     const bool last_pass = p.pass == kBoundPasses - 1;
+    const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 w2 = make_float2(inv_w, inv_w);
     uint32_t tile = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -297,14 +323,25 @@ __global__ void __launch_bounds__(BoundConfig<D>::kThreads, 1)
       const bool valid_row = t < p.n_q;
       const int64_t o = static_cast<int64_t>(h) * p.n_q + (valid_row ? t : 0);
       const int lo_idx = valid_row ? p.st.lo_idx[o] : 0;
-      const float lo_f = static_cast<float>(lo_idx);  // exact: lo_idx < 2^21
-      const float hi_f = first_pass ? 3.0e38f : static_cast<float>(kBoundBins);
-      const float x_off = valid_row ? -p.lse_dense[o] * 1.4426950408889634f : 0.f;
+      const int need_in = valid_row ? p.st.need[o] : 0;
+      // need < 0: fewer values above 2^-64 than B, so all of them are in the top B
+      const bool take_all = need_in < 0;
+      // y = s * scale_log2 + (64 - lse * log2 e): the same rounding in every pass
+      const float y_off = (valid_row ? -p.lse_dense[o] * 1.4426950408889634f : 0.f) - kBoundLo;
+      const float2 off2 = make_float2(y_off, y_off);
+      // Interval of this pass in y: [lo_idx, lo_idx + 32) / inv_w (exact: powers of two, lo_idx < 2^21).
+      // y is held below 64 (the top cell of every pass keeps a value at or above 2^0 by rounding).
+      const float lo_f = static_cast<float>(lo_idx);
+      const float y_top = (lo_f + static_cast<float>(kBoundBins)) / inv_w;  // the interval's top
+      const float y_in = lo_f / inv_w;              // the interval's bottom
+      // cell - 1 = floor(y * inv_w - lo_idx) = bits(y * inv_w + 1.5 * 2^23 - lo_idx, rounded down) - bits(1.5 * 2^23)
+      const float magic = 12582912.0f - lo_f;   // exact integer
+      const float2 magic2 = make_float2(magic, magic);
+
 #pragma unroll 4
-      for (int bb = 0; bb < kBoundBins; ++bb) {
-        hn[bb * 32] = 0u;
-        hm[bb * 32] = 0.f;
-      }
+      for (int bb = 0; bb < kBoundSubs * kBoundCells; ++bb) *reinterpret_cast<uint16_t*>(my_hist + bb * kCellBytes) = 0u;
+      float above = 0.f;   // last pass: P summed over the values above the interval
+      const float y_above = take_all ? 0.f : y_top;  // take_all: every value above 2^-64
       for (int j = 0; j < p.nkb; ++j, ++tile) {
         const uint32_t b = tile & 1u;
         const int n_valid = (j == p.nkb - 1) ? static_cast<int>(p.n_kv - static_cast<int64_t>(j) * 128) : 128;
@@ -321,69 +358,116 @@ __global__ void __launch_bounds__(BoundConfig<D>::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&s_free[b]);  // S is in registers: the buffer may be overwritten
-        // tb = grid coordinate inside the interval: (x + 64) * 2^(5p-1) is exact, and
-        // subtracting the integer lo_idx is exact wherever the result can be in [0, 32).
-        // Values above the interval (tb >= 32) were counted by an earlier pass; in pass 0 they
-        // are values above 2^0 by a rounding and go to the top bin. The in-interval test of
-        // all 64 values comes first (no votes); then one warp-uniform test per group of 8
-        // values skips the groups no lane needs (most of them after pass 0), and inside a
-        // group the histogram update is predicated, not branched per lane.
-        uint32_t in_mask[2] = {0u, 0u};
+        if (cols < 64) {  // a ragged last KV block: invalid columns become -inf (below every interval)
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = fmaf(__uint_as_float(r[c][e]), p.scale_log2, x_off);  // log2 P
-            const float tb = (x - kBoundLo) * inv_w - lo_f;
-            if ((32 * c + e < cols) && tb >= 0.f && tb < hi_f) in_mask[c] |= 1u << e;
-          }
+            for (int e = 0; e < 32; ++e)
+              if (32 * c + e >= cols) r[c][e] = 0xFF800000u;
+        }
+        if (!last_pass) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (!__any_sync(0xFFFFFFFFu, ((in_mask[c] >> (8 * g)) & 0xFFu) != 0u)) continue;
+            for (int e0 = 0; e0 < 32; e0 += kBoundSubs) {
+              // value e0 + u goes to histogram u: the four loads, then the four stores
+              // cell = bin + 1 = bits(tm) - bits(1.5 * 2^23) + 1; a value below the interval by more
+              // than a bin gives a smaller (or negative) tm, whose difference wraps above 33
+              uint32_t off[kBoundSubs];
 #pragma unroll
-            for (int e = 8 * g; e < 8 * g + 8; ++e) {
-              const bool in = (in_mask[c] >> e) & 1u;
-              const float x = fmaf(__uint_as_float(r[c][e]), p.scale_log2, x_off);
-              const float tb = (x - kBoundLo) * inv_w - lo_f;
-              const int bin = in ? min(static_cast<int>(tb), kBoundBins - 1) : 0;
-              hn[bin * 32] += in ? 1u : 0u;
-              hm[bin * 32] += in ? ex2_approx(x) : 0.f;
+              for (int u = 0; u < kBoundSubs; u += 2) {
+                const int e = e0 + u;
+                float2 yy = __ffma2_rn(make_float2(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), scale2, off2);
+                yy = make_float2(fminf(yy.x, kBoundYTop), fminf(yy.y, kBoundYTop));
+                const float2 tm = __ffma2_rd(yy, w2, magic2);
+                const uint32_t c0 = min(__float_as_uint(tm.x) - (kBoundMagicBits - 1u), kBoundCells - 1u);
+                const uint32_t c1 = min(__float_as_uint(tm.y) - (kBoundMagicBits - 1u), kBoundCells - 1u);
+                off[u] = c0 * kCellBytes + u * kSubBytes;
+                off[u + 1] = c1 * kCellBytes + (u + 1) * kSubBytes;
+              }
+              uint32_t cnt[kBoundSubs];
+#pragma unroll
+              for (int u = 0; u < kBoundSubs; ++u) cnt[u] = *reinterpret_cast<const uint16_t*>(my_hist + off[u]);
+#pragma unroll
+              for (int u = 0; u < kBoundSubs; ++u) *reinterpret_cast<uint16_t*>(my_hist + off[u]) = static_cast<uint16_t>(cnt[u] + 1u);
             }
           }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float yv[8];
+              bool any_in = false;
+#pragma unroll
+              for (int e2 = 0; e2 < 8; e2 += 2) {
+                const int e = 8 * g + e2;
+                const float2 yy = __ffma2_rn(make_float2(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), scale2, off2);
+                yv[e2] = fminf(yy.x, kBoundYTop);
+                yv[e2 + 1] = fminf(yy.y, kBoundYTop);
+                const float2 xx = __fadd2_rn(yy, make_float2(kBoundLo, kBoundLo));  // log2 P
+                above += (yv[e2] >= y_above ? ex2_approx(xx.x) : 0.f) + (yv[e2 + 1] >= y_above ? ex2_approx(xx.y) : 0.f);
+                any_in |= (yv[e2] >= y_in && yv[e2] < y_top) | (yv[e2 + 1] >= y_in && yv[e2 + 1] < y_top);
+              }
+              if (!__any_sync(0xFFFFFFFFu, any_in && !take_all)) continue;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const bool in = !take_all && yv[e] >= y_in && yv[e] < y_top;
+                const int bi = in ? static_cast<int>(__float_as_uint(__fmaf_rd(yv[e], inv_w, magic)) - kBoundMagicBits) : 0;
+                hn32[bi * 32] += in ? 1u : 0u;
+                hm[bi * 32] += in ? ex2_approx(yv[e] + kBoundLo) : 0.f;
+              }
+            }
+          }
+        }
       }
       // Both halves of every row are binned: combine and move the interval. The two warps of
       // a lane quarter reach both named barriers on every path (an aborted wait only ends
       // the tile loop early), so neither can be left waiting at one.
+      if (last_pass && half == 1) above_part[row] = above;
       asm volatile("bar.sync %0, %1;" ::"r"(1 + wq), "r"(64) : "memory");
       if (ok && half == 0 && valid_row) {
-        const uint32_t* hn2 = hn + 4 * kBoundBins * 32;
-        const float* hm2 = hm + 4 * kBoundBins * 32;
-        int need = p.st.need[o];
-        float above = p.st.above_sum[o];
-        int new_lo = lo_idx;
-        float rest = 0.f;  // last pass: the boundary bin's mean times the values still missing
-        int bin = kBoundBins - 1;
-        for (; bin >= 0; --bin) {
-          const int nb = static_cast<int>(hn[bin * 32] + hn2[bin * 32]);
-          const float mb = hm[bin * 32] + hm2[bin * 32];
-          if (nb >= need) {
-            rest = need > 0 ? mb * (static_cast<float>(need) / static_cast<float>(nb)) : 0.f;
-            break;
+        // the partner warp (w + 4) of this lane quarter binned the row's other 64 columns
+        const uint8_t* other = my_hist + 4 * C::kWarpHistBytes;
+        const uint32_t* hn32_2 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(hn32) + 4 * C::kWarpHistBytes);
+        const float* hm2 = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(hm) + 4 * C::kWarpHistBytes);
+        int need = need_in;
+        if (!last_pass) {
+          if (need > 0) {
+            int bin = kBoundBins - 1;
+            for (; bin >= 0; --bin) {  // bin b of the interval is cell b + 1
+              int nb = 0;
+              for (int u = 0; u < kBoundSubs; ++u) {
+                const uint32_t at = u * kSubBytes + (bin + 1) * kCellBytes;
+                nb += *reinterpret_cast<const uint16_t*>(my_hist + at) + *reinterpret_cast<const uint16_t*>(other + at);
+              }
+              if (nb >= need) break;
+              need -= nb;
+            }
+            if (bin >= 0) {
+              p.st.lo_idx[o] = (lo_idx + bin) * kBoundBins;  // that bin, in the next pass's widths
+              p.st.need[o] = need;
+            } else {
+              p.st.need[o] = -1;  // only reachable in pass 0: fewer values above 2^-64 than B
+            }
           }
-          need -= nb;
-          above += mb;
-        }
-        if (bin >= 0) {
-          new_lo = (lo_idx + bin) * kBoundBins;  // that bin, in the next pass's widths
         } else {
-          need = 0;  // fewer values above 2^-64 than B: all of them are in the top B
+          float u = above + above_part[row];
+          if (!take_all && need == 0) u = 0.f;  // an empty mask (B = 0) bounds nothing
+          if (!take_all && need > 0) {
+            for (int bin = kBoundBins - 1; bin >= 0; --bin) {
+              const int nb = static_cast<int>(hn32[bin * 32] + hn32_2[bin * 32]);
+              const float mb = hm[bin * 32] + hm2[bin * 32];
+              if (nb >= need) {  // the boundary bin's mean stands in for its top `need` values
+                u += mb * (static_cast<float>(need) / static_cast<float>(nb));
+                break;
+              }
+              need -= nb;
+              u += mb;
+            }
+          }
+          p.st.u[o] = u;
         }
-        p.st.lo_idx[o] = new_lo;
-        p.st.need[o] = need;
-        p.st.above_sum[o] = above;
-        if (last_pass || need == 0) p.st.u[o] = above + rest;
       }
       asm volatile("bar.sync %0, %1;" ::"r"(1 + wq), "r"(64) : "memory");  // histograms reused next item
     }

@@ -421,6 +421,55 @@ __global__ void __launch_bounds__(ScoreConfig<D>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------ scores across scales
+
+// Latent grid of a scale's current tokens, raster order (frame, row, column).
+struct GridDims {
+  int64_t t, h, w;
+};
+
+// Block of the previous scale's grid that holds the nearest raster position of block b of the
+// current grid: b's middle token c = start + (n - 1) / 2 is unravelled on `now`, each axis x of
+// size X' goes to the old cell (2x + 1) X / (2 X') (clipped to X - 1), and the old token is
+// ravelled on `prev` and divided by the block size. All integer arithmetic.
+__device__ __forceinline__ int64_t raster_block(int64_t b, int64_t n_now, const GridDims& now, const GridDims& prev,
+                                                int block) {
+  const int64_t s = b * block;
+  const int64_t e = min(s + block, n_now);
+  const int64_t c = s + (e - s - 1) / 2;
+  const int64_t hw = now.h * now.w;
+  const int64_t t = c / hw, rem = c - t * hw;
+  const int64_t h = rem / now.w, w = rem - h * now.w;
+  const int64_t to = min(prev.t - 1, (2 * t + 1) * prev.t / (2 * now.t));
+  const int64_t ho = min(prev.h - 1, (2 * h + 1) * prev.h / (2 * now.h));
+  const int64_t wo = min(prev.w - 1, (2 * w + 1) * prev.w / (2 * now.w));
+  return ((to * prev.h + ho) * prev.w + wo) / block;
+}
+
+constexpr int kMapRowsPerCta = 8;
+
+// S_now[h, i, j] = S_prev[h, m(i), c(j)] with m = raster_block (query blocks are current-scale
+// blocks) and c(j) = j on the KV prefix (text and reference blocks, the same tokens at every
+// scale), n_prefix + m(j - n_prefix) on the current-scale blocks. grid = (ceil(nqb_now / 8),
+// heads), 256 threads; the column map (nkb_now ints) is built once per CTA in shared memory.
+__global__ void __launch_bounds__(256) map_scores_kernel(const float* __restrict__ s_prev, float* __restrict__ s_now,
+                                                         int nqb_prev, int nkb_prev, int nqb_now, int nkb_now,
+                                                         int n_prefix, int64_t n_now, GridDims now, GridDims prev) {
+  extern __shared__ int col_map[];
+  for (int j = threadIdx.x; j < nkb_now; j += blockDim.x)
+    col_map[j] = j < n_prefix ? j : n_prefix + static_cast<int>(raster_block(j - n_prefix, n_now, now, prev, 128));
+  __syncthreads();
+  const int h = blockIdx.y;
+  const int i0 = blockIdx.x * kMapRowsPerCta;
+  const int i1 = min(nqb_now, i0 + kMapRowsPerCta);
+  for (int i = i0; i < i1; ++i) {
+    const int mi = static_cast<int>(raster_block(i, n_now, now, prev, 128));
+    const float* src = s_prev + (static_cast<int64_t>(h) * nqb_prev + mi) * nkb_prev;
+    float* dst = s_now + (static_cast<int64_t>(h) * nqb_now + i) * nkb_now;
+    for (int j = threadIdx.x; j < nkb_now; j += blockDim.x) dst[j] = __ldg(src + col_map[j]);
+  }
+}
+
 // ------------------------------------------------------------------------ Top-K
 
 // Order-preserving key: larger score -> larger key; -0.0 maps like +0.0; NaN ranks last.

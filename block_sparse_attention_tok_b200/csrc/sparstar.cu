@@ -40,6 +40,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxCandidates = 16384;  // Top-K keys held in shared memory (64 KB)
+constexpr int64_t kMaxMapColumns = 49152;  // columns of a mapped score row (192 KB column map)
 // Columns of each 128-column S row whose exp2 runs on the FMA pipe instead of MUFU.
 #ifndef SPARSTAR_POLY_COLS
 #define SPARSTAR_POLY_COLS 0
@@ -112,6 +113,8 @@ int set_kernel_attrs(DeviceInfo* d) {
                              ScoreConfig<64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMaxCandidates * 4)) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(map_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kMaxMapColumns * 4)) == cudaSuccess;
   if (!ok) return SPARSTAR_ERR_CUDA;
   // The attention kernels raise the softmax warps' registers with setmaxnreg, drawing on the
   // block's launch allocation; a build that launched with fewer registers would wait there
@@ -504,7 +507,8 @@ int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, i
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return SPARSTAR_ERR_WORKSPACE;
   const int64_t nqb = ceil_blocks(n_q), nkb = ceil_blocks(n_kv);
-  if (static_cast<int64_t>(heads) * nqb > INT32_MAX / 2 || n_q > INT32_MAX || n_kv > INT32_MAX || nqb > 65535 * 64LL)
+  if (static_cast<int64_t>(heads) * nqb > INT32_MAX / 2 || n_q > INT32_MAX || n_kv > INT32_MAX || nqb > 65535 * 64LL ||
+      nkb > kBoundMaxKvBlocks)
     return SPARSTAR_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
@@ -606,6 +610,41 @@ int sparstar_select_noalloc(const void* q, const void* k, int heads, int64_t n_q
   }
   return sparstar_select(q, k, heads, n_q, seg, head_dim, clip, density, budget_mode, idx, cnt, kmax, nullptr,
                          scratch, SPARSTAR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int sparstar_map_scores(const float* scores_prev, int heads, sparstar_segments seg_prev, sparstar_grid grid_prev,
+                        sparstar_segments seg_now, sparstar_grid grid_now, float* scores_now, void* stream) {
+  if (heads < 1 || heads > 65535 || !valid_segments(seg_prev) || !valid_segments(seg_now)) return SPARSTAR_ERR_ARG;
+  const sparstar_grid* grids[2] = {&grid_prev, &grid_now};
+  const int64_t n_cur[2] = {seg_prev.n_cur, seg_now.n_cur};
+  for (int g = 0; g < 2; ++g) {
+    const sparstar_grid& G = *grids[g];
+    if (G.frames < 1 || G.height < 1 || G.width < 1) return SPARSTAR_ERR_ARG;
+    const __int128 n = static_cast<__int128>(G.frames) * G.height * G.width;
+    if (n != n_cur[g]) return SPARSTAR_ERR_ARG;  // the grid lays out exactly the current tokens
+  }
+  if (seg_prev.n_text != seg_now.n_text || seg_prev.n_ctx != seg_now.n_ctx ||
+      seg_now.n_text % SPARSTAR_BLOCK != 0 || seg_now.n_ctx % SPARSTAR_BLOCK != 0)
+    return SPARSTAR_ERR_ARG;
+  const int64_t n_prefix = (seg_now.n_text + seg_now.n_ctx) / SPARSTAR_BLOCK;
+  const int64_t nqb_prev = ceil_blocks(seg_prev.n_cur), nqb_now = ceil_blocks(seg_now.n_cur);
+  const int64_t nkb_prev = n_prefix + nqb_prev, nkb_now = n_prefix + nqb_now;
+  if (nkb_now > kMaxMapColumns || nkb_prev > INT32_MAX || static_cast<int64_t>(heads) * nqb_prev * nkb_prev > (1LL << 40))
+    return SPARSTAR_ERR_UNSUPPORTED;
+  if (scores_prev == nullptr || scores_now == nullptr || (reinterpret_cast<uintptr_t>(scores_prev) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(scores_now) & 3u) != 0)
+    return SPARSTAR_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != SPARSTAR_OK) return rc;
+  if ((rc = set_kernel_attrs(dev)) != SPARSTAR_OK) return rc;
+  const GridDims now{grid_now.frames, grid_now.height, grid_now.width};
+  const GridDims prev{grid_prev.frames, grid_prev.height, grid_prev.width};
+  const dim3 grid(static_cast<unsigned>((nqb_now + kMapRowsPerCta - 1) / kMapRowsPerCta), static_cast<unsigned>(heads));
+  map_scores_kernel<<<grid, 256, static_cast<size_t>(nkb_now) * 4, static_cast<cudaStream_t>(stream)>>>(
+      scores_prev, scores_now, static_cast<int>(nqb_prev), static_cast<int>(nkb_prev), static_cast<int>(nqb_now),
+      static_cast<int>(nkb_now), static_cast<int>(n_prefix), seg_now.n_cur, now, prev);
+  return launch_status();
 }
 
 int sparstar_read_probe(const void* src, size_t bytes, unsigned* sink, void* stream) {

@@ -35,6 +35,10 @@ class Segments(ctypes.Structure):
     _fields_ = [("n_text", ctypes.c_int64), ("n_ctx", ctypes.c_int64), ("n_cur", ctypes.c_int64)]
 
 
+class Grid(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int64), ("height", ctypes.c_int64), ("width", ctypes.c_int64)]
+
+
 class Plan(ctypes.Structure):
     _fields_ = [("nqb", ctypes.c_int64), ("nkb", ctypes.c_int64), ("n_forced", ctypes.c_int64),
                 ("n_cand", ctypes.c_int64), ("k_total", ctypes.c_int32), ("k_topk", ctypes.c_int32)]
@@ -87,6 +91,8 @@ _SIGNATURES.update({
     "sparstar_topk": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _c.c_void_p, _c.c_void_p,
                                  _c.c_int32, _c.c_void_p]),
     "sparstar_read_probe": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_void_p, _c.c_void_p]),
+    "sparstar_map_scores": (_c.c_int, [_c.c_void_p, _c.c_int, Segments, Grid, Segments, Grid, _c.c_void_p,
+                                       _c.c_void_p]),
 })
 NOALLOC_SCRATCH_BYTES = 128 << 20
 
@@ -316,6 +322,24 @@ def select_noalloc(q: torch.Tensor, k: torch.Tensor, n_text: int, n_ctx: int, n_
                                           float(density), int(budget_mode), _ptr(idx), _ptr(cnt), idx.shape[-1],
                                           _stream_ptr(stream)), "sparstar_select_noalloc")
     return idx, cnt
+
+
+def map_scores(scores_prev: torch.Tensor, seg_prev, grid_prev, seg_now, grid_now, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Block scores of a previous scale of the clip carried to the current scale through the
+    nearest-raster-position block map (seg_* = (n_text, n_ctx, n_cur), grid_* = (frames, height,
+    width) of the current tokens). Returns fp32 [H, nqb_now, nkb_now]."""
+    if scores_prev.dtype != torch.float32 or not scores_prev.is_cuda or not scores_prev.is_contiguous() \
+            or scores_prev.dim() != 3:
+        raise ValueError("scores_prev must be a contiguous fp32 CUDA tensor [H, nqb, nkb]")
+    H = scores_prev.shape[0]
+    n_prefix = (seg_now[0] + seg_now[1]) // BLOCK
+    nqb_now = -(-seg_now[2] // BLOCK)
+    if out is None:
+        out = torch.empty(H, nqb_now, n_prefix + nqb_now, dtype=torch.float32, device=scores_prev.device)
+    _check(load().sparstar_map_scores(_ptr(scores_prev), H, Segments(*seg_prev), Grid(*grid_prev), Segments(*seg_now),
+                                      Grid(*grid_now), _ptr(out), _stream_ptr(stream)), "sparstar_map_scores")
+    return out
 
 
 def read_probe(buf: torch.Tensor, sink: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

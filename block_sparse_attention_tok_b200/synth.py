@@ -46,6 +46,7 @@ class Scale:
     clip: int          # 1 = first clip (ctx is the image pyramid), >= 2 = later clip (ctx is the preceding clip's final scale)
     density: float
     layers: int = 1
+    grid: Optional[Tuple[int, int, int]] = None   # (frames, height, width) of the current tokens
 
     @property
     def n_kv(self) -> int:
@@ -67,11 +68,15 @@ FINAL_CLIP1_RAGGED = Scale("final720p_clip1_72000_ragged", heads=32, head_dim=12
                            n_text=512, n_ctx=8192, n_cur=72000, clip=1, density=0.09375)
 FINAL_CLIP2 = Scale("final720p_clip2_72192", heads=32, head_dim=128, n_q=72192, n_text=512,
                     n_ctx=72192, n_cur=72192, clip=2, density=0.09375)
-# Full refined-scale schedule of one clip: 36 layers x 32 heads at four scales.
+# Full refined-scale schedule of one clip: 36 layers x 32 heads at four scales. The pages give
+# the token counts' scale (about 72,000 at the 720p final scale) but no latent grid shapes; the
+# grids here (8 latent frames, growing height x width) only lay the synthetic current tokens out
+# in raster order for the cross-scale block map.
 SCHEDULE_CLIP1: Tuple[Scale, ...] = tuple(
     Scale(f"schedule_clip1_s{i + 1}_{n}", heads=32, head_dim=128, n_q=n, n_text=512, n_ctx=8192,
-          n_cur=n, clip=1, density=dens, layers=36)
-    for i, (n, dens) in enumerate(((8192, 0.625), (18432, 0.1875), (36864, 0.1875), (72192, 0.09375)))
+          n_cur=n, clip=1, density=dens, layers=36, grid=grid)
+    for i, (n, dens, grid) in enumerate(((8192, 0.625, (8, 32, 32)), (18432, 0.1875, (8, 48, 48)),
+                                         (36864, 0.1875, (8, 64, 72)), (72192, 0.09375, (8, 94, 96))))
 )
 
 WORKLOADS = {s.name: s for s in (TINY_CLIP2, MID_CLIP1, FINAL_CLIP1_RAGGED, FINAL_CLIP2) + SCHEDULE_CLIP1}

@@ -213,6 +213,35 @@ int sparstar_forward_ex(const void* q, const void* k, const void* v, int heads, 
 int sparstar_retained_mass(const float* lse_kept, const float* lse_dense, int heads,
                            int64_t n_q, float* r_token, float* e_block, void* stream);
 
+/* Latent grid of a scale's current-scale tokens in raster order (frame, row, column):
+ * frames * height * width == n_cur. */
+typedef struct sparstar_grid {
+    int64_t frames;
+    int64_t height;
+    int64_t width;
+} sparstar_grid;
+
+/* Mask reuse across scales (digest, 关键结果与论文证据, bullet 重算频率, Figure 5: the mask
+ * recomputed at every scale, every second scale, or once and transferred). Carries the block
+ * scores of a previous scale of the same clip (from sparstar_select with `scores`) to the
+ * current scale, so that sparstar_topk can fill the current scale's rows without new scores:
+ *   scores_now[h][i][j] = scores_prev[h][m(i)][c(j)],
+ * with m(b) the previous-scale block that holds the nearest raster position of current block b
+ * (b's middle token c = 128 b + (n_b - 1) / 2 on grid_now, each axis x of size X' moved to the
+ * cell (2x + 1) X / (2 X') of grid_prev, clipped to X - 1, and ravelled back), and c(j) = j for
+ * the text and reference blocks (the same tokens at every scale) and n_prefix + m(j - n_prefix)
+ * for the current-scale blocks. Query blocks are current-scale blocks. The pages give no block
+ * correspondence between scales; this nearest-position map is this library's reading.
+ * scores_prev fp32 [H, ceil(n_cur_prev/128), n_prefix + ceil(n_cur_prev/128)] device,
+ * scores_now fp32 [H, ceil(n_cur_now/128), n_prefix + ceil(n_cur_now/128)] device (written),
+ * n_prefix = (n_text + n_ctx) / 128. Requirements: 1 <= heads <= 65535; grids of positive
+ * sizes whose products equal each scale's n_cur; equal n_text and n_ctx in both scales, each a
+ * multiple of 128 (else SPARSTAR_ERR_ARG); n_prefix + ceil(n_cur_now/128) <= 49152 (else
+ * SPARSTAR_ERR_UNSUPPORTED). Exact: a gather, no arithmetic on the scores. */
+int sparstar_map_scores(const float* scores_prev, int heads, sparstar_segments seg_prev,
+                        sparstar_grid grid_prev, sparstar_segments seg_now, sparstar_grid grid_now,
+                        float* scores_now, void* stream);
+
 /* Device bytes of the workspace of sparstar_token_bound: four [H,Nq] arrays of 4 bytes. */
 int sparstar_token_bound_workspace_size(int heads, int64_t n_q, size_t* bytes);
 
@@ -228,7 +257,8 @@ int sparstar_token_bound_workspace_size(int heads, int64_t n_q, size_t* bytes);
  * lse_dense fp32 [H,Nq] (natural log, from sparstar_attn with every block kept);
  * sm_scale <= 0 selects 1/sqrt(d). u_token: fp32 [H,Nq] device or NULL; u_block: fp32
  * [H,nqb] device. workspace: device, >= sparstar_token_bound_workspace_size() bytes,
- * 256-byte aligned. Requires an sm_100 device. n_q == 0 is a no-op. */
+ * 256-byte aligned. ceil(n_kv/128) <= 4095 (the counting passes keep 16-bit counts; else
+ * SPARSTAR_ERR_UNSUPPORTED). Requires an sm_100 device. n_q == 0 is a no-op. */
 int sparstar_token_bound(const void* q, const void* k, int heads, int64_t n_q, int64_t n_kv,
                          int head_dim, const int32_t* idx, const int32_t* cnt, int32_t kmax,
                          const float* lse_dense, float sm_scale, float* u_token, float* u_block,

@@ -173,3 +173,34 @@ def test_read_probe_rejects_bad_arguments_before_launch(lib):
     assert lib.sparstar_read_probe(0x1000, 40, 0x2000, None) == sparstar.ERR_ARG       # not a multiple of 16
     assert lib.sparstar_read_probe(0x1000, 64, None, None) == sparstar.ERR_ARG         # no sink
     assert lib.sparstar_read_probe(0x1000, 0, None, None) == sparstar.OK               # empty: no-op
+
+
+def test_map_scores_rejects_bad_arguments_before_launch(lib):
+    seg = sparstar.Segments
+    grid = sparstar.Grid
+    ok_args = (0x1000, 2, seg(256, 512, 384), grid(2, 8, 24), seg(256, 512, 768), grid(2, 12, 32), 0x2000, None)
+
+    def call(**over):
+        names = ["sp", "H", "seg_p", "grid_p", "seg_n", "grid_n", "sn", "st"]
+        a = dict(zip(names, ok_args))
+        a.update(over)
+        return lib.sparstar_map_scores(*(a[n] for n in names))
+
+    assert call(H=0) == sparstar.ERR_ARG
+    assert call(grid_p=grid(2, 8, 25)) == sparstar.ERR_ARG                        # product != n_cur
+    assert call(grid_n=grid(0, 12, 32)) == sparstar.ERR_ARG                        # empty axis
+    assert call(seg_n=seg(128, 512, 768)) == sparstar.ERR_ARG                      # text differs across scales
+    assert call(seg_p=seg(200, 512, 384), seg_n=seg(200, 512, 768)) == sparstar.ERR_ARG   # prefix not whole blocks
+    assert call(sp=None) == sparstar.ERR_ARG
+    assert call(sn=0x2002) == sparstar.ERR_ARG                                    # not 4-byte aligned
+    big = 49152 * 128
+    assert call(seg_n=seg(256, 512, big), grid_n=grid(1, 128, 49152)) == sparstar.ERR_UNSUPPORTED
+
+
+def test_token_bound_rejects_too_many_kv_blocks_before_launch(lib):
+    ws = ctypes.c_size_t()
+    assert lib.sparstar_token_bound_workspace_size(1, 128, ctypes.byref(ws)) == sparstar.OK
+    n_kv = 128 * 4096                     # 4,096 KV blocks: one more than the 16-bit counts allow
+    rc = lib.sparstar_token_bound(0x1000, 0x2000, 1, 128, n_kv, 128, 0x3000, 0x4000, 4, 0x5000, 0.0, None,
+                                  0x6000, 0x7000, ws.value, None)
+    assert rc == sparstar.ERR_UNSUPPORTED
