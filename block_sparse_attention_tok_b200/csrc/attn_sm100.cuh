@@ -187,32 +187,11 @@ __device__ __forceinline__ float row_max(const uint32_t (&r)[NC][32]) {
   return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// 2^x on the FMA pipe for a pair of arguments x <= 8: n = round(x) with the 1.5*2^23
-// shifter, f = x - n in [-1/2, 1/2], 2^f by a degree-3 polynomial (coefficients from
-// tests/exp2_poly_fit.py: Chebyshev-node least squares of the relative error, max 1.2e-4), and
-// 2^n added into the exponent field. Arguments below -125 are clamped there (2^-125 is
-// far below anything a bf16 P or the fp32 row sum can register).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c1 = 0.6933686137199402f, c2 = 0.24221783876419067f, c3 = 0.05459282547235489f;
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
-  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  q = __ffma2_rn(q, f, make_float2(c1, c1));
-  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
-template <int D, int kPolyCols, int B = 128>
+template <int D, int B = 128>
 __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
     attn_sparse_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnConfig<D, B>;
-  static_assert(kPolyCols % 32 == 0 && kPolyCols <= C::kCols, "software exp2 works on whole 32-column chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -506,13 +485,7 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[c][2 * e]), __uint_as_float(r[c][2 * e + 1])),
                                         scale2, neg_m2);
-            float2 pr;
-            if (c >= C::kSC - kPolyCols / 32) {
-              pr = exp2_poly2(x);
-            } else {
-              pr.x = ex2_approx(x.x);
-              pr.y = ex2_approx(x.y);
-            }
+            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
             acc[e & 3] = __fadd2_rn(acc[e & 3], pr);
             pk[e] = pack_bf16x2(pr.x, pr.y);
           }

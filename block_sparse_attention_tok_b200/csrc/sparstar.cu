@@ -41,12 +41,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxCandidates = 16384;  // Top-K keys held in shared memory (64 KB)
 constexpr int64_t kMaxMapColumns = 49152;  // columns of a mapped score row (192 KB column map)
-// Columns of each 128-column S row whose exp2 runs on the FMA pipe instead of MUFU.
-#ifndef SPARSTAR_POLY_COLS
-#define SPARSTAR_POLY_COLS 0
-#endif
-constexpr int kPolyCols128 = SPARSTAR_POLY_COLS;
-constexpr int kPolyCols64 = SPARSTAR_POLY_COLS;
 
 struct DeviceInfo {
   bool ready = false;
@@ -95,13 +89,13 @@ int set_kernel_attrs(DeviceInfo* d) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (d->attrs_set) return SPARSTAR_OK;
   bool ok = true;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128, kPolyCols128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<128>::kSmemBytes) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, kPolyCols64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64>::kSmemBytes) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128, 0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<128, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<128, 64>::kSmemBytes) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, 0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok &= cudaFuncSetAttribute(attn_sparse_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnConfig<64, 64>::kSmemBytes) == cudaSuccess;
   ok &= cudaFuncSetAttribute(bound_pass_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BoundConfig<128>::kSmemBytes) == cudaSuccess;
@@ -123,10 +117,10 @@ int set_kernel_attrs(DeviceInfo* d) {
     cudaFuncAttributes a;
     return cudaFuncGetAttributes(&a, kernel) == cudaSuccess && a.numRegs * threads >= needed;
   };
-  if (!regs_ok(attn_sparse_kernel<128, kPolyCols128>, AttnConfig<128>::kThreads, AttnConfig<128>::kRegsNeeded) ||
-      !regs_ok(attn_sparse_kernel<64, kPolyCols64>, AttnConfig<64>::kThreads, AttnConfig<64>::kRegsNeeded) ||
-      !regs_ok(attn_sparse_kernel<128, 0, 64>, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kRegsNeeded) ||
-      !regs_ok(attn_sparse_kernel<64, 0, 64>, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kRegsNeeded))
+  if (!regs_ok(attn_sparse_kernel<128>, AttnConfig<128>::kThreads, AttnConfig<128>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<64>, AttnConfig<64>::kThreads, AttnConfig<64>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<128, 64>, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kRegsNeeded) ||
+      !regs_ok(attn_sparse_kernel<64, 64>, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kRegsNeeded))
     return SPARSTAR_ERR_UNSUPPORTED;
   d->attrs_set = true;
   return SPARSTAR_OK;
@@ -456,14 +450,14 @@ int sparstar_attn_ex(const void* q, const void* k, const void* v, int heads, int
   const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
   if (block == 128) {
     if (head_dim == 128)
-      attn_sparse_kernel<128, kPolyCols128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
+      attn_sparse_kernel<128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
     else
-      attn_sparse_kernel<64, kPolyCols64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
+      attn_sparse_kernel<64><<<grid, AttnConfig<64>::kThreads, AttnConfig<64>::kSmemBytes, st>>>(tq, tk, tv, p);
   } else {
     if (head_dim == 128)
-      attn_sparse_kernel<128, 0, 64><<<grid, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
+      attn_sparse_kernel<128, 64><<<grid, AttnConfig<128, 64>::kThreads, AttnConfig<128, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
     else
-      attn_sparse_kernel<64, 0, 64><<<grid, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
+      attn_sparse_kernel<64, 64><<<grid, AttnConfig<64, 64>::kThreads, AttnConfig<64, 64>::kSmemBytes, st>>>(tq, tk, tv, p);
   }
   return launch_status();
 }
