@@ -437,6 +437,9 @@ def run_ours(args, rank, world, local_rank):
     if args.heads:
         sc_full = dataclasses.replace(sc_full, heads=args.heads)
     if args.scaling == "strong":
+        # every rank takes the same decision here, before any collective, so none is left waiting
+        if world > sc_full.heads:
+            raise SystemExit(f"{sc_full.heads} heads cannot be split over {world} ranks: every rank needs a head")
         # this rank's heads of the one input (the same bytes the one-rank run draws for them)
         h0, h1 = shard.head_range(rank, world, sc_full.heads)
         q, k, v = shard.make_shard_inputs(sc_full, rank, world, device=dev)
@@ -445,8 +448,6 @@ def run_ours(args, rank, world, local_rank):
         q, k, v = synth.make_qkv(sc_full.n_q, sc_full.n_kv, sc_full.heads, sc_full.head_dim,
                                  rank_seeds(sc_full, rank), device=dev)
     sc = dataclasses.replace(sc_full, heads=h1 - h0)   # what this rank computes
-    if sc.heads < 1:
-        raise SystemExit(f"rank {rank}: no heads to run ({sc_full.heads} heads over {world} ranks)")
     plan = S.make_plan(sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.clip, sc.density, args.budget_mode)
     kmax = int(plan.k_total)
     ws = S.Workspace(sc.heads, sc.n_q, sc.n_text, sc.n_ctx, sc.n_cur, sc.head_dim, dev)
