@@ -66,7 +66,8 @@ def parse():
     return ap.parse_args()
 
 
-ATTN_SOURCES = ("attn_sm100.cuh", "ptx.cuh")   # the attention kernel's device code
+# the attention kernel's device code and the host code that picks its launch (grid size)
+ATTN_SOURCES = ("attn_sm100.cuh", "ptx.cuh", "sparstar.cu")
 
 
 def kernel_source_hash(sources=ATTN_SOURCES) -> str:
