@@ -454,6 +454,13 @@ __global__ void __launch_bounds__(AttnConfig<D, B>::kThreads, 1)
         }
         ++tiles;
         tc_fence_after();
+        if (B < C::kRows && wq * 32 >= B) {
+          // 64-token blocks: rows B..127 of the MMA tile belong to no query block and are never
+          // stored, so their warps release P (whatever S left there) without a softmax
+          tc_fence_before();
+          mbar_arrive(&p_full[s]);
+          continue;
+        }
         uint32_t r[C::kSC][32];
 #pragma unroll
         for (int c = 0; c < C::kSC; ++c) tmem_ld32(t_s + 32 * c, r[c]);

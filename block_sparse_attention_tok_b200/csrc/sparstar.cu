@@ -45,7 +45,6 @@ constexpr int64_t kMaxMapColumns = 49152;  // columns of a mapped score row (192
 struct DeviceInfo {
   bool ready = false;
   int major = 0, minor = 0, sms = 0;
-  int64_t l2_bytes = 0;
   unsigned* status = nullptr;
   bool attrs_set = false;
 };
@@ -69,7 +68,6 @@ int device_info(DeviceInfo** out) {
     d.major = prop.major;
     d.minor = prop.minor;
     d.sms = prop.multiProcessorCount;
-    d.l2_bytes = prop.l2CacheSize;
     void* sym = nullptr;
     if (cudaGetSymbolAddress(&sym, g_status) != cudaSuccess) return SPARSTAR_ERR_CUDA;
     d.status = static_cast<unsigned*>(sym);
@@ -210,23 +208,6 @@ void launch_topk(const float* S, int64_t rows, int nkb, int n_forced, int k_topk
       launch_after(topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(128),
                    static_cast<size_t>(nkb - n_forced) * 4, st, S, nkb, n_forced, k_topk, idx, cnt, kmax);
   }
-}
-
-// CTAs of the persistent attention kernel (two slots each). Items run head-major, so a head's
-// K/V stays in L2 while its query blocks are processed. When two heads' K/V would not fit in L2
-// together, the number of slots is chosen so that each wave of items covers an equal share of
-// one head instead of straddling two (e.g. 141 CTAs = 282 slots for 564 query blocks): the
-// K/V of only one head is live at a time.
-int attn_grid(const DeviceInfo* dev, int heads, int64_t nqb, int64_t n_kv, int head_dim) {
-  const int64_t items = static_cast<int64_t>(heads) * nqb;
-  const int64_t full = 2LL * dev->sms;
-  int64_t slots = items < full ? items : full;
-  const int64_t kv_head_bytes = 2LL * n_kv * head_dim * 2;
-  if (dev->l2_bytes > 0 && 2 * kv_head_bytes > dev->l2_bytes && nqb > full) {
-    const int64_t waves = (nqb + full - 1) / full;
-    slots = (nqb + waves - 1) / waves;
-  }
-  return static_cast<int>((slots + 1) / 2);
 }
 
 int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, unsigned box_rows = 128) {
@@ -465,7 +446,8 @@ int sparstar_attn_ex(const void* q, const void* k, const void* v, int heads, int
   const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int grid = attn_grid(dev, heads, nqb, n_kv, head_dim);
+  const int slots_needed = (p.n_items + 1) / 2;
+  const int grid = slots_needed < dev->sms ? slots_needed : dev->sms;
   if (block == 128) {
     if (head_dim == 128)
       attn_sparse_kernel<128><<<grid, AttnConfig<128>::kThreads, AttnConfig<128>::kSmemBytes, st>>>(tq, tk, tv, p);
