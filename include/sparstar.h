@@ -49,7 +49,8 @@ extern "C" {
 #endif
 
 #define SPARSTAR_BLOCK 128
-#define SPARSTAR_ABI_VERSION 1
+/* 2: adds sparstar_map_scores and sparstar_read_probe (every version-1 entry point unchanged). */
+#define SPARSTAR_ABI_VERSION 2
 
 /* Return codes. */
 #define SPARSTAR_OK 0

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strerror(lib):
-    assert lib.sparstar_abi_version() == 1
+    assert lib.sparstar_abi_version() == 2
     for code in range(7):
         assert sparstar.strerror(code)
     assert sparstar.strerror(99) == "unknown status"
