@@ -86,6 +86,63 @@ def test_attention_on_random_masks(S, d, n_q, n_kv):
     _attn_with_oracle_mask(S, q, k, v, rows)
 
 
+@pytest.mark.parametrize("block", [128, 64])
+@pytest.mark.parametrize("d,H,n_q,n_kv", [(64, 3, 128 * 37 + 5, 128 * 23 + 77), (128, 2, 128 * 41, 128 * 19 + 1)])
+def test_attention_with_uneven_row_counts(S, block, d, H, n_q, n_kv):
+    """The attention ABI takes a count per row: rows of 1 to nkb kept blocks (first, last and
+    ragged blocks among them) in one launch, with kmax above every count, so the persistent
+    slots carry items of very different lengths; every query block compared."""
+    q, k, v = synth.make_qkv(n_q, n_kv, H, d, [800 + 3 * h + block for h in range(H)], device="cuda")
+    nqb, nkb = O.num_blocks(n_q, block), O.num_blocks(n_kv, block)
+    kmax = nkb + 3
+    rng = np.random.default_rng(n_q + n_kv + block)
+    rows = np.full((H, nqb, kmax), -1, dtype=np.int32)
+    counts = rng.integers(1, nkb + 1, size=(H, nqb))
+    counts[0, 0], counts[-1, -1] = 1, nkb
+    for h in range(H):
+        for i in range(nqb):
+            rows[h, i, :counts[h, i]] = np.sort(rng.choice(nkb, counts[h, i], replace=False))
+    rows[0, 1, :1] = nkb - 1   # a row holding only the ragged last block
+    counts[0, 1] = 1
+    idx = torch.from_numpy(rows).cuda()
+    cnt = torch.from_numpy(counts.astype(np.int32)).cuda()
+    o, lse = S.attn(q, k, v, idx, cnt, block=block)
+    assert S.device_status() == S.OK
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    o_np, lse_np = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(H):
+        qf, kf, vf = _f64(qb[h]), _f64(kb[h]), _f64(vb[h])
+        rows_h = np.where(np.arange(kmax)[None, :] < counts[h][:, None], rows[h], -1)
+        for i, (o_ref, lse_ref) in enumerate(O.block_sparse_attention(qf, kf, vf, rows_h, range(nqb), block=block)):
+            s, e = O.block_token_range(i, n_q, block)
+            check_output(o_np[h, s:e], o_ref, f"h{h} qb{i}")
+            assert np.abs(lse_np[h, s:e] - lse_ref).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("world", [2, 3, 5])
+def test_head_shards_equal_the_whole(S, world):
+    """The head split of the multi-GPU path, on one GPU: each rank's slice (its own inputs,
+    drawn as make_shard_inputs draws them) run through selection + attention gives exactly the
+    rows, outputs and LSEs of those heads in the one-rank run (per-head masks, no exchange)."""
+    from block_sparse_attention_tok_b200 import shard
+    sc = synth.Scale("shard_check_clip2", heads=7, head_dim=128, n_q=128 * 9 + 40, n_text=256, n_ctx=1024,
+                     n_cur=128 * 9 + 40, clip=2, density=0.3)
+    q, k, v = synth.make_qkv(sc.n_q, sc.n_kv, sc.heads, sc.head_dim,
+                             [sc.seed(h, 0, 0, 0) for h in range(sc.heads)], device="cuda")
+    seg = (sc.n_text, sc.n_ctx, sc.n_cur)
+    o, lse, idx, cnt = S.forward(q, k, v, *seg, sc.clip, sc.density)
+    for rank in range(world):
+        h0, h1 = shard.head_range(rank, world, sc.heads)
+        if h0 == h1:
+            continue
+        qs, ks, vs = shard.make_shard_inputs(sc, rank, world, device="cuda")
+        assert torch.equal(qs, q[h0:h1]) and torch.equal(ks, k[h0:h1]) and torch.equal(vs, v[h0:h1])
+        o_r, lse_r, idx_r, cnt_r = S.forward(qs, ks, vs, *seg, sc.clip, sc.density)
+        assert torch.equal(idx_r, idx[h0:h1]) and torch.equal(cnt_r, cnt[h0:h1])
+        assert torch.equal(o_r, o[h0:h1]) and torch.equal(lse_r, lse[h0:h1])
+    assert S.device_status() == S.OK
+
+
 def test_many_items_per_slot(S):
     """More (head, query block) items than two per CTA slot: exercises the per-slot item
     sequence (Q buffer reuse, O handover between items) of the persistent kernel."""
