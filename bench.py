@@ -39,6 +39,7 @@ from block_sparse_attention_tok_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 HBM_SPEC_GBS = 7700.0   # HGX B200 nominal HBM3e bandwidth
+L2_BYTES = 126 * 1000 * 1000
 METRIC = "sparse-attn TFLOP/s on kept tiles & % of bf16 peak; select GB/s; µs per scale"
 
 
@@ -314,8 +315,17 @@ def workload_config(sc, args, world):
     return {"workload": sc.name, "heads": sc.heads, "head_dim": sc.head_dim, "n_q": sc.n_q,
             "kv": {"text": sc.n_text, "ctx": sc.n_ctx, "cur": sc.n_cur}, "clip": sc.clip,
             "density": sc.density, "budget": "literal" if args.budget_mode == 0 else "candidates",
-            "block": 128, "per_gpu": per_gpu,
-            "l2": "no flush: inputs 3.5 GB > 126 MB L2", "parallelism": par}
+            "block": 128, "per_gpu": per_gpu, "l2": l2_note(sc, world, args.scaling), "parallelism": par}
+
+
+def l2_note(sc, world, scaling):
+    """How the timed steps stand to the 126 MB L2: a rank's q, k, v either exceed it (no flush
+    needed between steps) or fit in it (then they are said to stay resident)."""
+    heads = -(-sc.heads // world) if scaling == "strong" else sc.heads
+    nbytes = heads * (sc.n_q + 2 * sc.n_kv) * sc.head_dim * 2
+    if nbytes > L2_BYTES:
+        return f"no flush: inputs {nbytes / 1e9:.2f} GB per rank > 126 MB L2"
+    return f"inputs {nbytes / 1e6:.1f} MB per rank fit in the 126 MB L2 (not flushed)"
 
 
 def run_schedule(S, dev, stream, layers: int = 36):

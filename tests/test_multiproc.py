@@ -128,3 +128,22 @@ def test_two_gloo_ranks_split_heads_and_gather_equals_one_rank():
         _, o_all, q_bits = out[r]
         assert np.array_equal(q_bits, q.view(torch.int16).numpy())   # shards hold the one-rank bytes
         assert np.array_equal(o_all, ref)                            # gathered heads == one-rank result
+
+
+def test_bench_gpus_n_starts_its_own_ranks():
+    """`bench.py --gpus 2` without a torchrun environment spawns two ranks itself; on the
+    reference arm (the CPU oracle) rank 0 alone prints one JSON line and the other rank exits 0."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+                        "--warmup", "0", "--workload", "tiny_clip2_d64"], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert "fit in the 126 MB L2" in line["config"]["l2"]
