@@ -12,7 +12,8 @@ starts its own N ranks.
 
 Prints one JSON line (rank 0). Timed region: barrier + synchronize, K steps bracketed by
 CUDA events on the launch stream, synchronize + barrier; the max over ranks is reported.
-Inputs (3.5 GB in total) are far larger than L2 (126 MB), so no flush is inserted.
+Inputs (q, k, v: 2.97 GB at the 720p scale) are far larger than L2 (126 MB), so no flush is
+inserted; the config's `l2` key states it for the run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--scaling strong|weak]
 """
