@@ -58,6 +58,42 @@ def test_plan_matches_oracle_budget(lib, n_q, n_text, n_ctx, n_cur, clip, densit
     assert (plan.k_total, plan.k_topk) == O.row_budget(nkb, n_forced, density, mode)
 
 
+def test_plan_matches_oracle_budget_on_random_shapes(lib):
+    """3,000 seeded shapes: segment lengths from 0 to 10^5 tokens (ragged and block-aligned),
+    both clip modes, densities drawn from the pages' values, dyadic fractions and arbitrary
+    reals in (0, 1], both budget readings and both block sizes; every plan field equals the
+    oracle's (integers, so exactly)."""
+    rng = np.random.default_rng(20261202)
+    pages = [0.625, 0.1875, 0.09375, 1.0, 0.25, 0.5]
+    for _ in range(3000):
+        block = int(rng.choice([128, 64]))
+        lens = []
+        for _k in range(3):
+            r = rng.random()
+            if r < 0.2:
+                lens.append(0)
+            elif r < 0.5:
+                lens.append(int(rng.integers(1, 400)) * block)
+            else:
+                lens.append(int(rng.integers(1, 100000)))
+        n_text, n_ctx, n_cur = lens
+        if n_text + n_ctx + n_cur == 0:
+            n_cur = 1
+        n_q = int(rng.integers(0, 100000))
+        clip = int(rng.choice([1, 2, 3]))
+        r = rng.random()
+        density = (float(rng.choice(pages)) if r < 0.4 else
+                   int(rng.integers(1, 1025)) / 1024.0 if r < 0.7 else float(1.0 - rng.random()))
+        mode = int(rng.integers(0, 2))
+        plan = sparstar.make_plan(n_q, n_text, n_ctx, n_cur, clip, density, mode, block=block)
+        nkb = O.num_blocks(n_text + n_ctx + n_cur, block)
+        n_forced = min(O.forced_block_count(n_text, n_ctx, clip, block), nkb)
+        case = (n_q, n_text, n_ctx, n_cur, clip, density, mode, block)
+        assert plan.nqb == O.num_blocks(n_q, block) and plan.nkb == nkb, case
+        assert plan.n_forced == n_forced and plan.n_cand == nkb - n_forced, case
+        assert (plan.k_total, plan.k_topk) == O.row_budget(nkb, n_forced, density, mode), case
+
+
 def test_workspace_size(lib):
     # pooled q and k as bf16 hi/lo pairs (2 x H*n_blocks*d x 2 B each) and fp32 scores
     # (H*nqb*nkb), each section 256-byte aligned
