@@ -65,7 +65,7 @@ def test_tiny_clip2_scale_all_rows(S):
     assert stats["identical"] == stats["rows"]
 
 
-@pytest.mark.parametrize("case", list(synth.random_small_cases(seed=4321, count=16)), ids=lambda c: c["name"])
+@pytest.mark.parametrize("case", list(synth.random_small_cases(seed=4321, count=48)), ids=lambda c: c["name"])
 def test_small_ragged_cases(S, case):
     c = case
     q, k, v = synth.make_qkv(c["n_q"], c["n_text"] + c["n_ctx"] + c["n_cur"], c["H"], c["d"],

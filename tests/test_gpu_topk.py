@@ -136,3 +136,18 @@ def test_topk_nan_versus_negative_infinity(S):
     s = np.array([[np.nan, -np.inf, np.nan, -np.inf, 1.0] * 60], dtype=np.float32)
     for k in (1, 60, 61, 120, 150, 299):
         _check(S, s, 0, k)
+
+
+def test_topk_random_sweep(S):
+    """60 seeded launches: random candidate counts (2 to 6,000, so every keys-per-lane instance
+    and the CTA-per-row kernel), forced prefixes of 0 to 40 columns, K anywhere in [1, n_cand),
+    and rows of different kinds mixed in one launch."""
+    rng = np.random.default_rng(977)
+    for _ in range(60):
+        n_cand = int(rng.integers(2, 6001))
+        n_forced = int(rng.integers(0, 41))
+        k_topk = int(rng.integers(1, n_cand))
+        rows = int(rng.integers(1, 40))
+        kinds = rng.choice(KINDS, size=rows)
+        s = np.concatenate([_scores(str(kd), rng, 1, n_forced + n_cand) for kd in kinds])
+        _check(S, s, n_forced, k_topk, kmax=n_forced + k_topk + int(rng.integers(0, 3)))
